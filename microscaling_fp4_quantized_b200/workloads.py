@@ -1,0 +1,113 @@
+"""Seeded synthetic workloads for the FP4 attention forward.
+
+This module holds no arithmetic of the method: it only names the workload shapes and
+draws the random inputs. Both the tests (for the CPU oracle and the CUDA path) and
+the benchmark take their inputs from here.
+
+Recipe (the shapes stand in for the pages' video-diffusion and LLM workloads; no
+dataset is involved):
+  * One CPU ``torch.Generator`` seeded with the workload's seed draws, in this order,
+    Q, K, V ~ N(0, 1) as float32 [B, H, N, D]; then the per-channel K bias
+    ~ N(0, sigma^2) with shape [B, H, 1, D] (shared across tokens); then, for the
+    outlier workload only, per head one channel index (max(1, round(0.01 * D))
+    channels, drawn by ``randperm`` per head) that is multiplied by 20 in both Q and K.
+  * The outlier scaling and the bias are applied in float32, then the three tensors
+    are cast (round to nearest even) to the workload's dtype.
+Because the generator runs on the CPU, the same seed gives the same tensors on any
+machine, with or without a GPU.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import List, Optional
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    N: int
+    D: int
+    causal: bool
+    dtype: torch.dtype
+    seed: int
+    bias_sigma: float
+    outliers: bool = False
+
+    @property
+    def sm_scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+    @property
+    def ops(self) -> float:
+        """Attention operations per forward: 4*B*H*N^2*D, halved when causal."""
+        o = 4.0 * self.B * self.H * self.N * self.N * self.D
+        return o / 2 if self.causal else o
+
+    def describe(self) -> dict:
+        return {"workload": self.name, "B": self.B, "H": self.H, "N": self.N, "D": self.D,
+                "causal": self.causal, "dtype": str(self.dtype).replace("torch.", ""),
+                "seed": self.seed, "k_bias_sigma": self.bias_sigma, "outlier_channels": self.outliers}
+
+
+def _sweep() -> List[Workload]:
+    out = []
+    idx = 0
+    for D in (64, 128):
+        for N in (1024, 4096, 16384, 65536):
+            for causal in (False, True):
+                B = max(1, 65536 // N)
+                out.append(Workload(f"sweep_D{D}_N{N}_{'causal' if causal else 'full'}", B, 32, N, D,
+                                    causal, torch.bfloat16, 4 + idx, 2.0))
+                idx += 1
+    return out
+
+
+TINY = Workload("tiny_B1_H2_N256_D64_fp16", 1, 2, 256, 64, False, torch.float16, 0, 2.0)
+MEDIUM = Workload("B1_H16_N4096_D128", 1, 16, 4096, 128, False, torch.bfloat16, 1, 2.0)
+LLM_CAUSAL = Workload("llm_causal_B4_H32_N8192_D128_outliers", 4, 32, 8192, 128, True,
+                      torch.bfloat16, 2, 2.0, outliers=True)
+LONG = Workload("video_long_B1_H24_N32768_D128", 1, 24, 32768, 128, False, torch.bfloat16, 3, 4.0)
+SWEEP = _sweep()
+
+ALL = [TINY, MEDIUM, LLM_CAUSAL, LONG] + SWEEP
+
+
+def by_name(name: str) -> Workload:
+    for w in ALL:
+        if w.name == name:
+            return w
+    raise KeyError(name)
+
+
+def custom(B: int, H: int, N: int, D: int, causal: bool = False, dtype=torch.bfloat16,
+           seed: int = 123, bias_sigma: float = 2.0, outliers: bool = False) -> Workload:
+    return Workload(f"custom_B{B}_H{H}_N{N}_D{D}_{'causal' if causal else 'full'}", B, H, N, D,
+                    causal, dtype, seed, bias_sigma, outliers)
+
+
+def make_inputs(w: Workload, device: Optional[str] = None):
+    """Draw (q, k, v) as [B, H, N, D] tensors of ``w.dtype`` (on ``device`` if given)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+    shape = (w.B, w.H, w.N, w.D)
+    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    k = torch.randn(shape, generator=g, dtype=torch.float32)
+    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    bias = torch.randn((w.B, w.H, 1, w.D), generator=g, dtype=torch.float32) * w.bias_sigma
+    if w.outliers:
+        count = max(1, int(round(0.01 * w.D)))
+        for b in range(w.B):
+            for h in range(w.H):
+                ch = torch.randperm(w.D, generator=g)[:count]
+                q[b, h, :, ch] *= 20.0
+                k[b, h, :, ch] *= 20.0
+    k += bias
+    q, k, v = q.to(w.dtype), k.to(w.dtype), v.to(w.dtype)
+    if device is not None:
+        q, k, v = q.to(device), k.to(device), v.to(device)
+    return q, k, v
