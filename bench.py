@@ -1,0 +1,322 @@
+"""Benchmark of the microscaling-FP4 attention forward on B200.
+
+One step = one whole forward (K mean + quantization of Q, K, V + fused FP4 attention) over
+one batch of the long-sequence workload (B=1, H=24, N=32768, D=128, bf16, non-causal).
+Metric: attention TOPS = 4*B*H*N^2*D (halved when causal) per second, whole job over all
+ranks. The inputs (576 MiB) exceed the 126 MB L2, so no flush runs between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Under torchrun each rank runs its own copy of the workload (independent problems: weak
+scaling, no data-path collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from microscaling_fp4_quantized_b200 import workloads  # noqa: E402
+
+METRIC = "FP4 attention fwd TOPS (4·B·H·N²·D/s) at N=32K D=128; % of B200 FP4 peak"
+UNIT = "TOPS"
+DEFAULT_WORKLOAD = workloads.LONG.name
+FP4_NOMINAL_TFLOPS = 9000.0
+FP4_PER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return j, "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) during the timed region."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = f"/tmp/sage_clocks_{os.getpid()}.csv"
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    smax.append(float(parts[1]))
+                    power.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[4:8]):
+                    if val.lower().startswith("active"):
+                        reasons.add(nm)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
+
+
+def cpu_oracle_rate(wl, budget_s: float, q=None, k=None, v=None):
+    """Time the CPU oracle (as it stands) on a bounded sample of the workload: one head's
+    quantization plus as many query rows as fit the budget; extrapolate to TOPS."""
+    import numpy as np
+    import oracle
+    oracle.build()
+    if q is None:
+        small = workloads.Workload(wl.name, 1, 1, wl.N, wl.D, wl.causal, wl.dtype, wl.seed, wl.bias_sigma,
+                                   wl.outliers)
+        q, k, v = workloads.make_inputs(small)
+    qh = q.reshape(-1, wl.N, wl.D)[:1].float().numpy()
+    kh = k.reshape(-1, wl.N, wl.D)[:1].float().numpy()
+    vh = v.reshape(-1, wl.N, wl.D)[:1].float().numpy()
+    t0 = time.perf_counter()
+    qz = oracle.quantize_qkv(qh, kh, vh)
+    t_quant = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    rows_done, t_rows, n = 0, 0.0, 8
+    ops_rows = 0.0
+    while t_rows < budget_s and rows_done < wl.N:
+        n = min(n, wl.N - rows_done)
+        idx = rng.choice(wl.N, size=n, replace=False)
+        rows = np.stack([np.zeros(n, np.int64), idx], 1)
+        t0 = time.perf_counter()
+        oracle.attn_emulated(qz, wl.causal, wl.sm_scale, Bk=128, rows=rows)
+        dt = time.perf_counter() - t0
+        t_rows += dt
+        rows_done += n
+        keys = (idx + 1) if wl.causal else np.full(n, wl.N)
+        ops_rows += float((4.0 * keys * wl.D).sum())
+        n = int(min(4 * n, max(8, n * (budget_s - t_rows) / max(dt, 1e-6))))
+    per_head_ops = 4.0 * wl.N * wl.N * wl.D / (2 if wl.causal else 1)
+    # time of a whole head = quantization + rows extrapolated by op count
+    t_head = t_quant + t_rows * per_head_ops / ops_rows
+    value = per_head_ops / t_head / 1e12
+    sample = (f"1 of {wl.B * wl.H} heads: quantize N={wl.N} x D={wl.D} ({t_quant:.2f} s) + "
+              f"{rows_done} query rows over all keys ({t_rows:.2f} s); extrapolated to the whole forward")
+    return value, t_quant + t_rows, sample, oracle.num_threads()
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    budget = 2.0
+    for _ in range(args.warmup):
+        cpu_oracle_rate(wl, 0.5)
+    vals, times = [], []
+    sample = ""
+    cores = 1
+    for _ in range(args.steps):
+        v, t, sample, cores = cpu_oracle_rate(wl, budget)
+        vals.append(v)
+        times.append(t)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.median(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": wl.describe(),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    args = ap.parse_args()
+    wl = workloads.by_name(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, wl)
+
+    import microscaling_fp4_quantized_b200 as sage
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    q, k, v = workloads.make_inputs(wl)          # CPU, seeded
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    out = torch.empty_like(qd)
+    plan = sage.Plan(wl.B, wl.H, wl.N, wl.D, wl.dtype, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev_mid=None, ev_end=None):
+        plan.quantize(qd, kd, vd)
+        if ev_mid is not None:
+            ev_mid.record(stream)
+        plan.attention(out, causal=wl.causal, sm_scale=wl.sm_scale)
+        if ev_end is not None:
+            ev_end.record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if sage.device_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    sampler = ClockSampler(local) if rank == 0 or True else None
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    mids = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_begin.record(stream)
+    for i in range(args.steps):
+        starts[i].record(stream)
+        step(mids[i], ends[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if dist is not None:
+        dist.barrier()
+    elapsed_ms = t_begin.elapsed_time(t_end)
+    attn_ms = [mids[i].elapsed_time(ends[i]) for i in range(args.steps)]
+    quant_ms = [starts[i].elapsed_time(mids[i]) for i in range(args.steps)]
+    if dist is not None:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+    value = world * wl.ops / (ms_per_step * 1e-3) / 1e12
+    err = sage.device_error()
+
+    # --- end to end through the public API: pinned host inputs -> result on the host ---
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+        oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+        e2e_steps = max(3, min(args.steps, 10))
+
+        def e2e_step():
+            a = qh.to(dev, non_blocking=True)
+            b = kh.to(dev, non_blocking=True)
+            c = vh.to(dev, non_blocking=True)
+            o = sage.attn(a, b, c, causal=wl.causal, sm_scale=wl.sm_scale)
+            oh.copy_(o, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1) / e2e_steps
+        if dist is not None:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        nbytes = q.numel() * q.element_size()
+        e2e = {"value": world * wl.ops / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes}
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, basis = _peaks()
+    sustained = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    fp4_peak = FP4_PER_BF16 * sustained
+    attn_avg_ms = statistics.mean(attn_ms)
+    achieved = wl.ops / (attn_avg_ms * 1e-3) / 1e12
+    roofline = {
+        "kernel": "attn_fp4_fwd_kernel", "bound": "tensor", "achieved": achieved, "peak": fp4_peak,
+        "unit": "TFLOP/s", "frac": achieved / fp4_peak, "traffic": None,
+        "peak_basis": f"{basis} bf16 sustained {sustained} TFLOP/s x {FP4_PER_BF16:g} (nominal FP4:BF16)",
+        "frac_of_nominal_9pflops": achieved / FP4_NOMINAL_TFLOPS,
+        "attn_ms": attn_avg_ms, "quant_ms": statistics.mean(quant_ms),
+    }
+    cpu = None
+    if not args.no_cpu_baseline:
+        val, _, sample, cores = cpu_oracle_rate(wl, args.cpu_budget_s)
+        cpu = {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+    cfg = wl.describe()
+    cfg["l2"] = "inputs larger than L2 (no flush)"
+    cfg["timing"] = "CUDA events on the launching stream, max over ranks"
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp4_e2m1", "data": "synthetic",
+        "config": cfg, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": 3 * args.steps, "clocks": clocks, "device_error_word": err,
+        "pct_of_fp4_peak": 100.0 * value / world / fp4_peak,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,150 @@
+/*
+ * sage_fp4.h -- C ABI of the B200 (sm_100a) microscaling-FP4 attention forward.
+ *
+ * The operation (SageAttention3, "Microscaling FP4 Attention for Inference ...",
+ * arXiv 2505.11594, abstract: plug-and-play FP4 attention on Blackwell FP4 tensor cores):
+ *
+ *   O = softmax(sm_scale * Q K^T [+ causal mask]) V        per (batch, head)
+ *
+ * computed as:
+ *   1. K smoothing: K' = K - mean_over_tokens(K) per (b, h, channel)  (SageAttention
+ *      OpenReview thread, reply to W1, "smoothing K"; softmax is invariant to it).
+ *   2. Q, K', V quantized to FP4 E2M1 with one unsigned E4M3 scale per 16 consecutive
+ *      elements (Q and K' along the head dimension, V along tokens).
+ *   3. S = Q^ K^^T as a block-scaled FP4 tensor-core contraction (FP32 accumulate),
+ *      FlashAttention tiling with the online softmax m/d recurrence (same thread, reply
+ *      to Q3), diag(l)^-1 applied after the last key tile (reply to Q2).
+ *   4. P~ quantized with two-level scaling: a per-row factor s1 = rowmax(P~)/(448*6)
+ *      per key tile, then the same 16-element E4M3/E2M1 rule; P^ V^ as a second
+ *      block-scaled FP4 contraction, accumulated in FP32.
+ *
+ * Conventions for every entry point
+ *   - Tensors are device pointers unless stated; the caller owns all memory. The
+ *     library keeps no per-call state and never frees caller memory.
+ *   - Q, K, V, O: [B, H, N, D] contiguous, element type bf16 or fp16 (sage_dtype_t).
+ *   - D must be 64 or 128; B, H, N >= 0 (any zero gives an empty problem: SAGE_OK,
+ *     nothing launched); N need not be a multiple of anything.
+ *   - All pointers must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call is
+ *     asynchronous on it; argument errors are returned before anything is launched.
+ *   - sm_scale <= 0 selects 1/sqrt(D).
+ *   - No C++ exception crosses this boundary.
+ *   - Every wait inside the kernels is bounded (default 2 s). A wait that runs out sets
+ *     a device error word, the kernel drains its own copies, frees its tensor memory
+ *     and returns; sage_fp4_get_device_error() reports it (SAGE_ERR_TIMEOUT).
+ *
+ * Quantized layouts (Np = N rounded up to a multiple of 128; rows/tokens >= N are 0):
+ *   q_fp4, k_fp4 : [B*H, Np, D/2] bytes. Byte j of row n holds elements 2j (low nibble)
+ *                  and 2j+1 (high nibble) of that row. E2M1 code = sign<<3 | magnitude.
+ *   vt_fp4       : [B*H, D, Np/2] bytes: V transposed; byte j of row d holds tokens 2j
+ *                  (low nibble) and 2j+1 (high nibble).
+ *   q_sf, k_sf   : [B*H, Np/128, D/64, 512] bytes, the tensor-core scale-factor tiling.
+ *                  The scale of (bh, token n, channels 16c..16c+15) is at
+ *                    ((bh*(Np/128) + n/128) * (D/64) + (16c)/64) * 512
+ *                    + (n%32)*16 + ((n%128)/32)*4 + c%4
+ *   vt_sf        : [B*H, Np/128, 2, 512] bytes. The scale of (bh, channel d, tokens
+ *                  16t..16t+15) is at
+ *                    ((bh*(Np/128) + (16t)/128) * 2 + ((16t)%128)/64) * 512
+ *                    + (d%32)*16 + (d/32)*4 + t%4
+ *                  (for D = 64 the bytes with d/32 >= 2 are 0).
+ *   k_mean       : [B*H, D] float32: fp32(sum_n K[bh, n, d] in binary64 / N).
+ */
+#ifndef SAGE_FP4_H
+#define SAGE_FP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SAGE_OK = 0,
+  SAGE_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, short workspace */
+  SAGE_ERR_UNSUPPORTED = 2, /* D not in {64, 128}, or a size beyond the 32-bit indexing limits */
+  SAGE_ERR_CUDA = 3,        /* a CUDA runtime/driver call or launch failed */
+  SAGE_ERR_TIMEOUT = 4      /* a bounded wait inside a kernel ran out (see above) */
+} sage_status_t;
+
+typedef enum { SAGE_BF16 = 0, SAGE_F16 = 1 } sage_dtype_t;
+
+/* Human-readable name of a status code (static storage). */
+const char* sage_status_string(sage_status_t status);
+
+/* Byte sizes of the quantized tensors for a problem (0 for an empty problem). */
+typedef struct {
+  size_t q_fp4, q_sf, k_fp4, k_sf, vt_fp4, vt_sf, k_mean;
+} sage_fp4_sizes_t;
+sage_status_t sage_fp4_quantized_sizes(int B, int H, int N, int D, sage_fp4_sizes_t* sizes);
+
+/* Scratch bytes sage_fp4_quantize_qkv needs (binary64 partial sums for the K mean). */
+size_t sage_fp4_quantize_scratch_bytes(int B, int H, int N, int D);
+
+/*
+ * Steps 1-2 alone: K mean, then quantize Q, K - mean (smooth_k != 0) or K (smooth_k == 0),
+ * and V^T into the layouts above. Outputs are written in full (padding included).
+ * scratch: device memory of at least sage_fp4_quantize_scratch_bytes(); contents are
+ * overwritten. k_mean may be NULL when smooth_k == 0.
+ */
+sage_status_t sage_fp4_quantize_qkv(const void* q, const void* k, const void* v, sage_dtype_t dtype,
+                                    int B, int H, int N, int D, int smooth_k, uint8_t* q_fp4,
+                                    uint8_t* q_sf, uint8_t* k_fp4, uint8_t* k_sf, uint8_t* vt_fp4,
+                                    uint8_t* vt_sf, float* k_mean, void* scratch,
+                                    size_t scratch_bytes, void* stream);
+
+/*
+ * Steps 3-4 on already-quantized inputs (layouts above): the fused tensor-core attention
+ * kernel. out: [B, H, N, D] of out_dtype. Uses no scratch memory.
+ */
+sage_status_t sage_fp4_attn_fwd_quantized(const uint8_t* q_fp4, const uint8_t* q_sf,
+                                          const uint8_t* k_fp4, const uint8_t* k_sf,
+                                          const uint8_t* vt_fp4, const uint8_t* vt_sf, void* out,
+                                          sage_dtype_t out_dtype, int B, int H, int N, int D,
+                                          int causal, float sm_scale, void* stream);
+
+/* Workspace bytes sage_fp4_attn_fwd_ex needs: the quantized tensors plus scratch. */
+size_t sage_fp4_workspace_bytes(int B, int H, int N, int D);
+
+/*
+ * The whole forward (steps 1-4) with a caller-owned workspace of at least
+ * sage_fp4_workspace_bytes() bytes (256-byte aligned). Three kernel launches.
+ */
+sage_status_t sage_fp4_attn_fwd_ex(const void* q, const void* k, const void* v, void* out,
+                                   sage_dtype_t dtype, int B, int H, int N, int D, int causal,
+                                   float sm_scale, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * The whole forward on bf16 tensors with a library-owned workspace taken from the
+ * stream-ordered allocator (cudaMallocAsync / cudaFreeAsync on `stream`).
+ */
+sage_status_t sage_fp4_attn_fwd(const void* q, const void* k, const void* v, void* out, int B,
+                                int H, int N, int D, int causal, float sm_scale, void* stream);
+
+/*
+ * S = sm_scale * Q^ K^^T (dequantized FP4 operands, FP32 accumulation) for every query
+ * and key of the quantized inputs: s_out is [B*H, Np, Np] float32. The tensor-core
+ * contraction of step 3 on its own, exported so that it can be checked in isolation.
+ */
+sage_status_t sage_fp4_qk_scores(const uint8_t* q_fp4, const uint8_t* q_sf, const uint8_t* k_fp4,
+                                 const uint8_t* k_sf, float* s_out, int B, int H, int N, int D,
+                                 float sm_scale, void* stream);
+
+/*
+ * Read and clear the device error word the kernels set when a bounded wait runs out.
+ * Synchronizes `stream`. *word receives the raw bits (0 = none); returns SAGE_OK when
+ * the word was 0, SAGE_ERR_TIMEOUT when a wait ran out, SAGE_ERR_CUDA on a CUDA error.
+ */
+sage_status_t sage_fp4_get_device_error(uint32_t* word, void* stream);
+
+/*
+ * Bound on every in-kernel wait, in nanoseconds (default 2e9; 0 restores the default).
+ * Applies to launches made after the call.
+ */
+sage_status_t sage_fp4_set_wait_timeout_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGE_FP4_H */

@@ -1,0 +1,587 @@
+// Fused microscaling-FP4 attention forward for B200 (sm_100a).
+//
+// Method: SageAttention3 (arXiv 2505.11594, abstract) -- FP4 Q, K, P~, V on the
+// Blackwell FP4 tensor cores -- with FlashAttention tiling and the online softmax
+// m/d recurrence as the SageAttention OpenReview thread states it (reply to Q3),
+// diag(l)^-1 after the last key tile (reply to Q2), and the two-level P~ quantization
+// (per-row factor s1 = rowmax(P~)/(448*6) per key tile, then 16-element E4M3 scales).
+//
+// One CTA per (128-query tile, batch*head); key tiles of 128. Warp roles:
+//   warp 0      TMA producer: Q^ + scales once, then K^/V^T tiles + scales into a
+//               3-stage shared-memory ring (cp.async.bulk.tensor / cp.async.bulk).
+//   warp 1      allocates 512 tensor-memory columns; one thread issues the tcgen05
+//               block-scaled MMAs: S = Q^ K^^T (kind::mxf4nvf4, M128 N128 K64 steps)
+//               into a double-buffered S in TMEM, and PV = P^ V^T (N = D) into TMEM.
+//   warps 2-5   softmax: thread r owns query row r; reads its S row from TMEM, applies
+//               the causal / length mask, updates the running max and sum, computes the
+//               per-tile row factor and the per-16 E4M3 scales, writes P^ codes
+//               (128B-row swizzle the MMA expects) and scale tiles to shared memory.
+//   warps 6-9   correction: O_row = O_row * alpha + s1 * PV_row in FP32 registers per
+//               tile, and the O / l epilogue.
+// Every mbarrier wait is bounded (globaltimer); a wait that runs out raises the CTA's
+// abort flag and the device error word, and all roles drain and return.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+#include "sage_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace sage {
+
+namespace {
+
+constexpr int kStages = 3;
+constexpr int kStatSlots = 4;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kAttnThreads = 320;
+
+constexpr int align1k(int x) { return (x + 1023) & ~1023; }
+
+// Tensor-memory column map of the attention kernel.
+constexpr uint32_t kColS0 = 0;      // S buffers: 128 columns each, at 0 and 128
+constexpr uint32_t kColPV = 256;    // PV accumulator: D columns
+constexpr uint32_t kColSfQ = 384;   // 4 columns per 64-wide K chunk of D
+constexpr uint32_t kColSfK = 392;   // + 8 * stage
+constexpr uint32_t kColSfV = 416;   // + 8 * stage
+constexpr uint32_t kColSfP = 440;   // + 8 * P buffer
+
+template <int D>
+struct Layout {
+  static constexpr int kQBytes = 128 * D / 2;
+  static constexpr int kSfQKBytes = (D / 64) * 512;
+  static constexpr int kKBytes = 128 * D / 2;
+  static constexpr int kVBytes = D * 64;
+  static constexpr int kSfVBytes = 1024;
+  static constexpr int kPBytes = 128 * 64;
+  static constexpr int kSfPBytes = 1024;
+  static constexpr int off_q = 0;
+  static constexpr int off_sfq = align1k(off_q + kQBytes);
+  static constexpr int st_k = 0;
+  static constexpr int st_sfk = align1k(kKBytes);
+  static constexpr int st_v = align1k(st_sfk + kSfQKBytes);
+  static constexpr int st_sfv = align1k(st_v + kVBytes);
+  static constexpr int kStageBytes = align1k(st_sfv + kSfVBytes);
+  static constexpr int off_stage = align1k(off_sfq + kSfQKBytes);
+  static constexpr int off_p = off_stage + kStages * kStageBytes;
+  static constexpr int off_sfp = off_p + 2 * kPBytes;
+  static constexpr int off_stats = off_sfp + 2 * kSfPBytes;  // [slot][3][128] floats
+  static constexpr int off_bar = off_stats + kStatSlots * 3 * 128 * 4;
+  static constexpr int kNumBars = 32;
+  static constexpr int off_misc = off_bar + kNumBars * 8;    // tmem base, abort flag
+  static constexpr int kBytes = off_misc + 16;
+};
+
+// Barrier indices.
+enum : int {
+  B_QFULL = 0,
+  B_KFULL = 1,                    // + stage
+  B_VFULL = B_KFULL + kStages,    // + stage
+  B_KVEMPTY = B_VFULL + kStages,  // + stage
+  B_SFULL = B_KVEMPTY + kStages,  // + buffer
+  B_SEMPTY = B_SFULL + 2,
+  B_PFULL = B_SEMPTY + 2,
+  B_PEMPTY = B_PFULL + 2,
+  B_PVFULL = B_PEMPTY + 2,
+  B_PVEMPTY = B_PVFULL + 1,
+  B_STFULL = B_PVEMPTY + 1,       // + slot
+  B_DRAIN = B_STFULL + kStatSlots,
+  B_COUNT = B_DRAIN + 1
+};
+static_assert(B_COUNT <= 32, "barrier area");
+
+struct Ctl {
+  volatile uint32_t* abort;
+  uint32_t* err;
+  uint64_t timeout_ns;
+};
+
+// Bounded wait: true when the phase with `parity` has completed, false on abort/timeout.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& c) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*c.abort) return false;
+    if (globaltimer_ns() - t0 > c.timeout_ns) {
+      *c.abort = 1u;
+      atomicOr(c.err, kDevErrTimeout);
+      return false;
+    }
+  }
+}
+
+// 32 columns from TMEM, with the wait::ld tied to the registers it produces.
+__device__ __forceinline__ void tmem_wait_regs(uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+        "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+        "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+        "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
+  // 32 rows x 16 bytes, 8-row core matrices 128 bytes apart, no swizzle.
+  return make_sdesc(saddr, 0, 128, kLayoutNone);
+}
+
+template <int D>
+__device__ __forceinline__ uint64_t qk_desc(uint32_t saddr) {
+  // Rows of D/2 bytes (K-major), 8-row groups D*4 bytes apart, swizzle = row width.
+  return make_sdesc(saddr, 16, 8 * (D / 2), D == 128 ? kLayoutSw64 : kLayoutSw32);
+}
+
+__device__ __forceinline__ uint64_t row64_desc(uint32_t saddr) {
+  return make_sdesc(saddr, 16, 512, kLayoutSw64);
+}
+
+__device__ __forceinline__ void store_out8(void* out, size_t idx, const float* v, int dtype) {
+  uint4 w;
+  uint32_t* ww = reinterpret_cast<uint32_t*>(&w);
+  if (dtype == kDtypeBF16) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+      ww[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+      ww[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+  }
+  *reinterpret_cast<uint4*>(static_cast<char*>(out) + idx * 2) = w;
+}
+
+}  // namespace
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_fp4_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + L::off_bar;
+  auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + L::off_misc);
+  float* stats = reinterpret_cast<float*>(smem + L::off_stats);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int nqt = p.Np / 128;
+  const int qt = CAUSAL ? (nqt - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
+  const int bh = blockIdx.y;
+  const int nt = CAUSAL ? (qt + 1) : nqt;  // key tiles to visit
+  Ctl ctl{misc + 1, p.err, p.timeout_ns};
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_QFULL), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(B_KFULL + s), 1);
+      mbar_init(bar(B_VFULL + s), 1);
+      mbar_init(bar(B_KVEMPTY + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(B_SFULL + b), 1);
+      mbar_init(bar(B_SEMPTY + b), 4);
+      mbar_init(bar(B_PFULL + b), 4);
+      mbar_init(bar(B_PEMPTY + b), 1);
+    }
+    mbar_init(bar(B_PVFULL), 1);
+    mbar_init(bar(B_PVEMPTY), 4);
+    for (int s = 0; s < kStatSlots; ++s) mbar_init(bar(B_STFULL + s), 4);
+    mbar_init(bar(B_DRAIN), 1);
+    misc[1] = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(sbase + L::off_misc, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer ----
+    if (lane == 0) {
+      const uint32_t sq = sbase + L::off_q;
+      mbar_arrive_expect_tx(bar(B_QFULL), L::kQBytes + L::kSfQKBytes);
+      tma_load_2d(sq, &tm_q, 0, bh * p.Np + qt * 128, bar(B_QFULL));
+      bulk_load(sbase + L::off_sfq, p.q_sf + (static_cast<size_t>(bh) * nqt + qt) * L::kSfQKBytes,
+                L::kSfQKBytes, bar(B_QFULL));
+      int issued = 0;
+      for (int j = 0; j < nt; ++j) {
+        const int st = j % kStages;
+        if (!wait_bar(bar(B_KVEMPTY + st), ((j / kStages) & 1) ^ 1, ctl)) break;
+        const uint32_t sst = sbase + L::off_stage + st * L::kStageBytes;
+        mbar_arrive_expect_tx(bar(B_KFULL + st), L::kKBytes + L::kSfQKBytes);
+        tma_load_2d(sst + L::st_k, &tm_k, 0, bh * p.Np + j * 128, bar(B_KFULL + st));
+        bulk_load(sst + L::st_sfk, p.k_sf + (static_cast<size_t>(bh) * nqt + j) * L::kSfQKBytes,
+                  L::kSfQKBytes, bar(B_KFULL + st));
+        mbar_arrive_expect_tx(bar(B_VFULL + st), L::kVBytes + L::kSfVBytes);
+        tma_load_2d(sst + L::st_v, &tm_v, j * 64, bh * D, bar(B_VFULL + st));
+        bulk_load(sst + L::st_sfv, p.vt_sf + (static_cast<size_t>(bh) * nqt + j) * L::kSfVBytes,
+                  L::kSfVBytes, bar(B_VFULL + st));
+        issued = j + 1;
+      }
+      if (*ctl.abort) {
+        // Let every copy this thread started land before the CTA releases its memory.
+        Ctl drain{misc + 2, p.err, p.timeout_ns};
+        misc[2] = 0u;
+        wait_bar(bar(B_QFULL), 0, drain);
+        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j) {
+          wait_bar(bar(B_KFULL + j % kStages), (j / kStages) & 1, drain);
+          wait_bar(bar(B_VFULL + j % kStages), (j / kStages) & 1, drain);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer ----
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = make_idesc_fp4(128);
+      constexpr uint32_t idesc_pv = make_idesc_fp4(D);
+      constexpr int kc_qk = D / 64;
+      bool ok = wait_bar(bar(B_QFULL), 0, ctl);
+      if (ok) {
+        tc_fence_after();
+        for (int c = 0; c < kc_qk; ++c)
+          tc_cp_sf(tmem + kColSfQ + 4 * c, sf_desc(sbase + L::off_sfq + 512 * c));
+      }
+      for (int j = 0; ok && j <= nt; ++j) {
+        if (j < nt) {
+          const int st = j % kStages, sb = j & 1;
+          const uint32_t sst = sbase + L::off_stage + st * L::kStageBytes;
+          if (!wait_bar(bar(B_KFULL + st), (j / kStages) & 1, ctl)) { ok = false; break; }
+          if (!wait_bar(bar(B_SEMPTY + sb), ((j >> 1) & 1) ^ 1, ctl)) { ok = false; break; }
+          tc_fence_after();
+          for (int c = 0; c < kc_qk; ++c)
+            tc_cp_sf(tmem + kColSfK + 8 * st + 4 * c, sf_desc(sst + L::st_sfk + 512 * c));
+          for (int c = 0; c < kc_qk; ++c)
+            tc_mma_fp4(tmem + kColS0 + 128 * sb, qk_desc<D>(sbase + L::off_q + 32 * c),
+                       qk_desc<D>(sst + L::st_k + 32 * c), idesc_s, tmem + kColSfQ + 4 * c,
+                       tmem + kColSfK + 8 * st + 4 * c, c > 0 ? 1u : 0u);
+          tc_commit(bar(B_SFULL + sb));
+        }
+        if (j >= 1) {
+          const int jj = j - 1;
+          const int st = jj % kStages, pb = jj & 1;
+          const uint32_t sst = sbase + L::off_stage + st * L::kStageBytes;
+          if (!wait_bar(bar(B_VFULL + st), (jj / kStages) & 1, ctl)) { ok = false; break; }
+          if (!wait_bar(bar(B_PFULL + pb), (jj >> 1) & 1, ctl)) { ok = false; break; }
+          if (!wait_bar(bar(B_PVEMPTY), (jj & 1) ^ 1, ctl)) { ok = false; break; }
+          tc_fence_after();
+          for (int c = 0; c < 2; ++c) {
+            tc_cp_sf(tmem + kColSfP + 8 * pb + 4 * c, sf_desc(sbase + L::off_sfp + pb * L::kSfPBytes + 512 * c));
+            tc_cp_sf(tmem + kColSfV + 8 * st + 4 * c, sf_desc(sst + L::st_sfv + 512 * c));
+          }
+          for (int c = 0; c < 2; ++c)
+            tc_mma_fp4(tmem + kColPV, row64_desc(sbase + L::off_p + pb * L::kPBytes + 32 * c),
+                       row64_desc(sst + L::st_v + 32 * c), idesc_pv, tmem + kColSfP + 8 * pb + 4 * c,
+                       tmem + kColSfV + 8 * st + 4 * c, c > 0 ? 1u : 0u);
+          tc_commit(bar(B_PVFULL));
+          tc_commit(bar(B_PEMPTY + pb));
+          tc_commit(bar(B_KVEMPTY + st));
+        }
+      }
+      // Drain: every MMA / copy issued above has completed before TMEM is released.
+      tc_commit(bar(B_DRAIN));
+      Ctl drain{misc + 3, p.err, p.timeout_ns};
+      misc[3] = 0u;
+      wait_bar(bar(B_DRAIN), 0, drain);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------- softmax ----
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int qrow = qt * 128 + r;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const float xs = p.sm_scale_log2;
+    float m_run = -INFINITY, l_run = 0.0f;
+    for (int j = 0; j < nt; ++j) {
+      const int sb = j & 1, pb = j & 1, slot = j % kStatSlots;
+      if (!__all_sync(0xffffffffu, wait_bar(bar(B_SFULL + sb), (j >> 1) & 1, ctl))) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + kColS0 + 128 * sb + 32 * c, sr[c]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_wait_regs(sr[c]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_SEMPTY + sb));
+
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(sr[c][i]);
+      const int kbase = j * 128;
+      const bool need_mask = CAUSAL ? (j == nt - 1) : (kbase + 128 > p.N);
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int key = kbase + c;
+          if (key >= p.N || (CAUSAL && key > qrow)) s[c] = -INFINITY;
+        }
+      }
+      float bm[8];
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        float m0 = s[16 * b];
+#pragma unroll
+        for (int i = 1; i < 16; ++i) m0 = fmaxf(m0, s[16 * b + i]);
+        bm[b] = m0;
+      }
+      float tm = bm[0];
+#pragma unroll
+      for (int b = 1; b < 8; ++b) tm = fmaxf(tm, bm[b]);
+      const float tmx = tm * xs;
+      const float m_new = fmaxf(m_run, tmx);
+      const float alpha = ex2_approx(m_run - m_new);
+      const float rfac = ex2_approx(tmx - m_new);  // rowmax of P~ in this tile
+      const float s1 = rfac * (1.0f / 2688.0f);
+
+      // Per-16 scales of P2 = P~ / s1 = exp2(S*xs - tmx) * 2688.
+      float inv[8];
+      uint32_t sfw0 = 0, sfw1 = 0;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        const float amax = ex2_approx(fmaf(bm[b], xs, -tmx)) * 2688.0f;
+        const uint32_t sbyte = f32_to_e4m3(amax * (1.0f / 6.0f));
+        const float sdec = e4m3_to_f32(sbyte);
+        inv[b] = sdec > 0.0f ? 2688.0f / sdec : 0.0f;
+        if (b < 4) sfw0 |= sbyte << (8 * b);
+        else sfw1 |= sbyte << (8 * (b - 4));
+      }
+      float rowsum = 0.0f;
+      uint32_t pw[16];
+#pragma unroll
+      for (int w = 0; w < 16; ++w) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const int k0 = 8 * w + 2 * h;
+          const float e0 = ex2_approx(fmaf(s[k0], xs, -tmx));
+          const float e1 = ex2_approx(fmaf(s[k0 + 1], xs, -tmx));
+          rowsum += e0 + e1;
+          const float iv = inv[k0 / 16];
+          word |= f32x2_to_e2m1(e0 * iv, e1 * iv) << (8 * h);
+        }
+        pw[w] = word;
+      }
+      l_run = l_run * alpha + rowsum * rfac;
+      m_run = m_new;
+
+      // P^ buffer pb must be free (PV of tile j-2 finished).
+      if (!__all_sync(0xffffffffu, wait_bar(bar(B_PEMPTY + pb), ((j >> 1) & 1) ^ 1, ctl))) break;
+      uint8_t* prow = smem + L::off_p + pb * L::kPBytes + r * 64;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int cs = c ^ ((r >> 1) & 3);
+        *reinterpret_cast<uint4*>(prow + cs * 16) = make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+      }
+      uint8_t* sfp = smem + L::off_sfp + pb * L::kSfPBytes + (r % 32) * 16 + (r / 32) * 4;
+      *reinterpret_cast<uint32_t*>(sfp) = sfw0;
+      *reinterpret_cast<uint32_t*>(sfp + 512) = sfw1;
+      fence_proxy_async_smem();
+      float* st = stats + slot * 3 * 128;
+      st[r] = alpha;
+      st[128 + r] = s1;
+      st[256 + r] = l_run;
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar(B_PFULL + pb));
+        mbar_arrive(bar(B_STFULL + slot));
+      }
+    }
+  } else {
+    // ---------------------------------------------------------- correction ----
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int qrow = qt * 128 + r;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    float o[D];
+#pragma unroll
+    for (int d = 0; d < D; ++d) o[d] = 0.0f;
+    float l_fin = 1.0f;
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      const int slot = j % kStatSlots;
+      if (!__all_sync(0xffffffffu, wait_bar(bar(B_STFULL + slot), (j / kStatSlots) & 1, ctl))) { ok = false; break; }
+      const float* st = stats + slot * 3 * 128;
+      const float alpha = st[r], s1 = st[128 + r];
+      l_fin = st[256 + r];
+      if (!__all_sync(0xffffffffu, wait_bar(bar(B_PVFULL), j & 1, ctl))) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + kColPV + 32 * c, v);
+        tmem_wait_regs(v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[32 * c + i] = fmaf(__uint_as_float(v[i]), s1, o[32 * c + i] * alpha);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_PVEMPTY));
+    }
+    if (ok && qrow < p.N) {
+      const float il = 1.0f / l_fin;
+      const size_t base = (static_cast<size_t>(bh) * p.N + qrow) * D;
+#pragma unroll
+      for (int d = 0; d < D; d += 8) {
+        float v8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v8[i] = o[d + i] * il;
+        store_out8(p.out, base + d, v8, p.out_dtype);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// S = sm_scale * Q^ K^^T for one (query tile, key tile, head): the QK^T stage alone.
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    qk_scores_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const AttnParams p) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  // Reuse the attention layout: Q tile at off_q, K tile in stage 0.
+  const uint32_t bar_full = sbase + L::off_bar, bar_mma = bar_full + 8;
+  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + L::off_misc);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int nqt = p.Np / 128;
+  const int qt = blockIdx.x, kt = blockIdx.y, bh = blockIdx.z;
+  Ctl ctl{misc + 1, p.err, p.timeout_ns};
+  constexpr uint32_t kCols = 256;
+  if (threadIdx.x == 0) {
+    mbar_init(bar_full, 1);
+    mbar_init(bar_mma, 1);
+    misc[1] = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sbase + L::off_misc, kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  const uint32_t sk = sbase + L::off_stage;
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_full, L::kQBytes + L::kKBytes + 2 * L::kSfQKBytes);
+      tma_load_2d(sbase + L::off_q, &tm_q, 0, bh * p.Np + qt * 128, bar_full);
+      tma_load_2d(sk + L::st_k, &tm_k, 0, bh * p.Np + kt * 128, bar_full);
+      bulk_load(sbase + L::off_sfq, p.q_sf + (static_cast<size_t>(bh) * nqt + qt) * L::kSfQKBytes, L::kSfQKBytes, bar_full);
+      bulk_load(sk + L::st_sfk, p.k_sf + (static_cast<size_t>(bh) * nqt + kt) * L::kSfQKBytes, L::kSfQKBytes, bar_full);
+      Ctl drain{misc + 2, p.err, p.timeout_ns};
+      misc[2] = 0u;
+      wait_bar(bar_full, 0, drain);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      if (wait_bar(bar_full, 0, ctl)) {
+        tc_fence_after();
+        constexpr int kc = D / 64;
+        for (int c = 0; c < kc; ++c) {
+          tc_cp_sf(tmem + 128 + 4 * c, sf_desc(sbase + L::off_sfq + 512 * c));
+          tc_cp_sf(tmem + 144 + 4 * c, sf_desc(sk + L::st_sfk + 512 * c));
+        }
+        for (int c = 0; c < kc; ++c)
+          tc_mma_fp4(tmem, qk_desc<D>(sbase + L::off_q + 32 * c), qk_desc<D>(sk + L::st_k + 32 * c),
+                     make_idesc_fp4(128), tmem + 128 + 4 * c, tmem + 144 + 4 * c, c > 0 ? 1u : 0u);
+      }
+      tc_commit(bar_mma);
+    }
+  } else {
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const bool ready = wait_bar(bar_mma, 0, ctl) && !*ctl.abort;
+    if (__all_sync(0xffffffffu, ready)) {
+      tc_fence_after();
+      float* out = static_cast<float*>(p.out) + (static_cast<size_t>(bh) * p.Np + qt * 128 + r) * p.Np + kt * 128;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + 32 * c, v);
+        tmem_wait_regs(v);
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(out + 32 * c + i) =
+              make_float4(__uint_as_float(v[i]) * p.sm_scale, __uint_as_float(v[i + 1]) * p.sm_scale,
+                          __uint_as_float(v[i + 2]) * p.sm_scale, __uint_as_float(v[i + 3]) * p.sm_scale);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kCols);
+  }
+}
+
+template <int D>
+static int attn_smem_bytes() {
+  const int need = Layout<D>::kBytes + 1024;
+  // At least 116 KiB so that two CTAs never share an SM (each holds all 512 TMEM columns).
+  return need > 116 * 1024 ? need : 116 * 1024;
+}
+
+template <int D, bool CAUSAL>
+static cudaError_t launch_attn_t(const TensorMaps& m, const AttnParams& p, cudaStream_t stream) {
+  const int smem = attn_smem_bytes<D>();
+  cudaError_t e = cudaFuncSetAttribute(attn_fp4_fwd_kernel<D, CAUSAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.Np / 128, p.BH);
+  attn_fp4_fwd_kernel<D, CAUSAL><<<grid, kAttnThreads, smem, stream>>>(m.q, m.k, m.v, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attention(const TensorMaps& m, const AttnParams& p, cudaStream_t stream) {
+  if (p.BH == 0 || p.N == 0) return cudaSuccess;
+  if (p.D == 64) return p.causal ? launch_attn_t<64, true>(m, p, stream) : launch_attn_t<64, false>(m, p, stream);
+  return p.causal ? launch_attn_t<128, true>(m, p, stream) : launch_attn_t<128, false>(m, p, stream);
+}
+
+template <int D>
+static cudaError_t launch_scores_t(const TensorMaps& m, const AttnParams& p, cudaStream_t stream) {
+  const int smem = Layout<D>::kBytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(qk_scores_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.Np / 128, p.Np / 128, p.BH);
+  qk_scores_kernel<D><<<grid, 192, smem, stream>>>(m.q, m.k, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_qk_scores(const TensorMaps& m, const AttnParams& p, cudaStream_t stream) {
+  if (p.BH == 0 || p.N == 0) return cudaSuccess;
+  return p.D == 64 ? launch_scores_t<64>(m, p, stream) : launch_scores_t<128>(m, p, stream);
+}
+
+}  // namespace sage
