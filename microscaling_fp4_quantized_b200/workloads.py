@@ -73,8 +73,10 @@ LLM_CAUSAL = Workload("llm_causal_B4_H32_N8192_D128_outliers", 4, 32, 8192, 128,
                       torch.bfloat16, 2, 2.0, outliers=True)
 LONG = Workload("video_long_B1_H24_N32768_D128", 1, 24, 32768, 128, False, torch.bfloat16, 3, 4.0)
 SWEEP = _sweep()
+# Profiling size: inputs (192 MiB) larger than the 126 MB L2, a few GB on the device at most.
+PROFILE = Workload("profile_B1_H16_N16384_D128", 1, 16, 16384, 128, False, torch.bfloat16, 7, 2.0)
 
-ALL = [TINY, MEDIUM, LLM_CAUSAL, LONG] + SWEEP
+ALL = [TINY, MEDIUM, LLM_CAUSAL, LONG, PROFILE] + SWEEP
 
 
 def by_name(name: str) -> Workload:
