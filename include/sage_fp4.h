@@ -122,6 +122,28 @@ sage_status_t sage_fp4_attn_fwd(const void* q, const void* k, const void* v, voi
                                 int H, int N, int D, int causal, float sm_scale, void* stream);
 
 /*
+ * The whole forward (steps 1-4) for callers that cannot allocate device memory. No
+ * passage of the method corresponds to it: it exists for callers that may not call
+ * cudaMalloc or any allocating library routine (engines that own a fixed memory pool,
+ * plugin hosts that forbid allocation while executing, threads without an initialised
+ * allocator). It allocates nothing: the caller passes q, k, v and out as for
+ * sage_fp4_attn_fwd_ex, and the scratch lives in a 16 MiB file-scope device array that
+ * every GPU which loads this library holds until the process exits.
+ *   - Limit: sage_fp4_workspace_bytes(B, H, N, D) must be <= 16 MiB (for example
+ *     B*H = 16, N = 4096, D = 128); larger problems return SAGE_ERR_UNSUPPORTED before
+ *     anything is launched.
+ *   - The first call on a device looks up the array's device address (with that device
+ *     current) and caches it; make that first call before any stream capture.
+ *   - Every call shares the one array, which keeps the last call's contents. Nothing in
+ *     it has to start at zero (each call writes every byte it later reads), but calls
+ *     that overlap on the GPU (different streams, or different host threads, on the same
+ *     device) race on it and corrupt each other's results: serialize them.
+ */
+sage_status_t sage_fp4_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
+                                        sage_dtype_t dtype, int B, int H, int N, int D, int causal,
+                                        float sm_scale, void* stream);
+
+/*
  * S = sm_scale * Q^ K^^T (dequantized FP4 operands, FP32 accumulation) for every query
  * and key of the quantized inputs: s_out is [B*H, Np, Np] float32. The tensor-core
  * contraction of step 3 on its own, exported so that it can be checked in isolation.

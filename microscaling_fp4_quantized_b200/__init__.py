@@ -30,7 +30,7 @@ EXPORTED = [
     "sage_status_string", "sage_fp4_quantized_sizes", "sage_fp4_quantize_scratch_bytes",
     "sage_fp4_quantize_qkv", "sage_fp4_attn_fwd_quantized", "sage_fp4_workspace_bytes",
     "sage_fp4_attn_fwd_ex", "sage_fp4_attn_fwd", "sage_fp4_qk_scores",
-    "sage_fp4_get_device_error", "sage_fp4_set_wait_timeout_ns",
+    "sage_fp4_get_device_error", "sage_fp4_set_wait_timeout_ns", "sage_fp4_attn_fwd_noalloc",
 ]
 
 
@@ -73,6 +73,7 @@ def lib():
         L.sage_fp4_qk_scores.argtypes = [u8p, u8p, u8p, u8p, vp, i, i, i, i, f, vp]
         L.sage_fp4_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), vp]
         L.sage_fp4_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+        L.sage_fp4_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
         for n in EXPORTED[1:]:
             if n not in ("sage_fp4_quantize_scratch_bytes", "sage_fp4_workspace_bytes"):
                 getattr(L, n).restype = i  # sage_status_t
@@ -194,6 +195,20 @@ def attn_bf16_library_workspace(q, k, v, causal: bool = False, sm_scale: Optiona
     _check(lib().sage_fp4_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, D,
                                    int(bool(causal)), float(sm_scale or 0.0), _stream(q.device)),
            "sage_fp4_attn_fwd")
+    return out
+
+
+def attn_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+                 sm_scale: Optional[float] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The forward through the entry point that allocates no device memory (its scratch is
+    a fixed 16 MiB device array inside the library; larger problems raise). For callers
+    that cannot allocate; calls on different streams of one device must not overlap."""
+    B, H, N, D = _check_qkv(q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().sage_fp4_attn_fwd_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q.dtype), B, H, N, D, int(bool(causal)),
+        float(sm_scale or 0.0), _stream(q.device)), "sage_fp4_attn_fwd_noalloc")
     return out
 
 
