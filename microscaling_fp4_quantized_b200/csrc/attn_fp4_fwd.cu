@@ -12,12 +12,13 @@
 //   warp 1      allocates 512 tensor-memory columns; one thread issues the tcgen05
 //               block-scaled MMAs: S = Q^ K^^T (kind::mxf4nvf4, M128 N128 K64 steps)
 //               into a double-buffered S in TMEM, and PV = P^ V^T (N = D) into TMEM.
-//   warps 2-5   softmax: thread r owns query row r; reads its S row from TMEM, applies
-//               the causal / length mask, updates the running max and sum, computes the
-//               per-tile row factor and the per-16 E4M3 scales, writes P^ codes
-//               (128B-row swizzle the MMA expects) and scale tiles to shared memory.
-//   warps 6-9   correction: O_row = O_row * alpha + s1 * PV_row in FP32 registers per
-//               tile, and the O / l epilogue.
+//   warps 2-9   two softmax/correction warpgroups. Thread (h, r) owns keys 64h..64h+63
+//               of query row r in every S tile and output channels [h*D/2, (h+1)*D/2)
+//               of that row. The two halves of a row exchange their maxima through
+//               shared memory; each half then computes P~, its per-16 E4M3 scales, the
+//               P^ codes (written in the swizzled layout the MMA reads) and its part of
+//               the row sum; and folds the previous tile's PV into its FP32 registers:
+//               O = O * alpha + s1 * PV.
 // Every mbarrier wait is bounded (globaltimer); a wait that runs out raises the CTA's
 // abort flag and the device error word, and all roles drain and return.
 #include <cuda_bf16.h>
@@ -33,7 +34,7 @@ namespace sage {
 namespace {
 
 constexpr int kStages = 3;
-constexpr int kStatSlots = 4;
+constexpr int kSoftmaxWarps = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kAttnThreads = 320;
 
@@ -66,8 +67,9 @@ struct Layout {
   static constexpr int off_stage = align1k(off_sfq + kSfQKBytes);
   static constexpr int off_p = off_stage + kStages * kStageBytes;
   static constexpr int off_sfp = off_p + 2 * kPBytes;
-  static constexpr int off_stats = off_sfp + 2 * kSfPBytes;  // [slot][3][128] floats
-  static constexpr int off_bar = off_stats + kStatSlots * 3 * 128 * 4;
+  static constexpr int off_xch = off_sfp + 2 * kSfPBytes;  // [2 tiles][2 halves][128] floats
+  static constexpr int off_lsum = off_xch + 2 * 2 * 128 * 4;  // [2 halves][128] floats
+  static constexpr int off_bar = off_lsum + 2 * 128 * 4;
   static constexpr int kNumBars = 32;
   static constexpr int off_misc = off_bar + kNumBars * 8;    // tmem base, abort flag
   static constexpr int kBytes = off_misc + 16;
@@ -85,8 +87,9 @@ enum : int {
   B_PEMPTY = B_PFULL + 2,
   B_PVFULL = B_PEMPTY + 2,
   B_PVEMPTY = B_PVFULL + 1,
-  B_STFULL = B_PVEMPTY + 1,       // + slot
-  B_DRAIN = B_STFULL + kStatSlots,
+  B_XCH = B_PVEMPTY + 1,          // + tile parity: row-max exchange between the halves
+  B_LSUM = B_XCH + 2,             // final row-sum exchange
+  B_DRAIN = B_LSUM + 1,
   B_COUNT = B_DRAIN + 1
 };
 static_assert(B_COUNT <= 32, "barrier area");
@@ -172,7 +175,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t bar0 = sbase + L::off_bar;
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + L::off_misc);
-  float* stats = reinterpret_cast<float*>(smem + L::off_stats);
+  float* xch = reinterpret_cast<float*>(smem + L::off_xch);
+  float* lsum = reinterpret_cast<float*>(smem + L::off_lsum);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int nqt = p.Np / 128;
@@ -190,13 +194,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(B_SFULL + b), 1);
-      mbar_init(bar(B_SEMPTY + b), 4);
-      mbar_init(bar(B_PFULL + b), 4);
+      mbar_init(bar(B_SEMPTY + b), kSoftmaxWarps);
+      mbar_init(bar(B_PFULL + b), kSoftmaxWarps);
       mbar_init(bar(B_PEMPTY + b), 1);
+      mbar_init(bar(B_XCH + b), kSoftmaxWarps);
     }
     mbar_init(bar(B_PVFULL), 1);
-    mbar_init(bar(B_PVEMPTY), 4);
-    for (int s = 0; s < kStatSlots; ++s) mbar_init(bar(B_STFULL + s), 4);
+    mbar_init(bar(B_PVEMPTY), kSoftmaxWarps);
+    mbar_init(bar(B_LSUM), kSoftmaxWarps);
     mbar_init(bar(B_DRAIN), 1);
     misc[1] = 0u;
     fence_mbar_init();
@@ -303,52 +308,91 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       misc[3] = 0u;
       wait_bar(bar(B_DRAIN), 0, drain);
     }
-  } else if (warp < 6) {
-    // ------------------------------------------------------------- softmax ----
+  } else {
+    // ------------------------------------------- softmax + correction (2 x 4 warps) ----
+    constexpr int DH = D / 2;
+    const int h = (warp - 2) >> 2;  // which half of the keys / output channels
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int qrow = qt * 128 + r;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const float xs = p.sm_scale_log2;
-    float m_run = -INFINITY, l_run = 0.0f;
-    for (int j = 0; j < nt; ++j) {
-      const int sb = j & 1, pb = j & 1, slot = j % kStatSlots;
-      if (!__all_sync(0xffffffffu, wait_bar(bar(B_SFULL + sb), (j >> 1) & 1, ctl))) break;
+    float o[DH];
+#pragma unroll
+    for (int d = 0; d < DH; ++d) o[d] = 0.0f;
+    float m_run = -INFINITY, l_half = 0.0f, alpha_prev = 1.0f, s1_prev = 0.0f;
+    bool ok = true;
+
+    // O = O * alpha + s1 * PV for this thread's DH output channels (PV of tile jj).
+    auto correct = [&](int jj, float alpha, float s1) -> bool {
+      if (!__all_sync(0xffffffffu, wait_bar(bar(B_PVFULL), jj & 1, ctl))) return false;
       tc_fence_after();
-      uint32_t sr[4][32];
+      const bool unit = __all_sync(0xffffffffu, alpha == 1.0f);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + kColS0 + 128 * sb + 32 * c, sr[c]);
+      for (int c = 0; c < DH / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + kColPV + DH * h + 32 * c, v);
+        tmem_wait_regs(v);
+        const float2 s12 = make_float2(s1, s1), a2 = make_float2(alpha, alpha);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_wait_regs(sr[c]);
+        for (int i = 0; i < 32; i += 2) {
+          float2 acc = make_float2(o[32 * c + i], o[32 * c + i + 1]);
+          if (!unit) acc = mul2(acc, a2);
+          acc = fma2(make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), s12, acc);
+          o[32 * c + i] = acc.x;
+          o[32 * c + i + 1] = acc.y;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_PVEMPTY));
+      return true;
+    };
+
+    for (int j = 0; j < nt; ++j) {
+      const int sb = j & 1, pb = j & 1;
+      if (!__all_sync(0xffffffffu, wait_bar(bar(B_SFULL + sb), (j >> 1) & 1, ctl))) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[2][32];
+      tmem_ld32(tmem + lane_base + kColS0 + 128 * sb + 64 * h, sr[0]);
+      tmem_ld32(tmem + lane_base + kColS0 + 128 * sb + 64 * h + 32, sr[1]);
+      tmem_wait_regs(sr[0]);
+      tmem_wait_regs(sr[1]);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_SEMPTY + sb));
 
-      float s[128];
+      float s[64];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 2; ++c)
 #pragma unroll
         for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(sr[c][i]);
-      const int kbase = j * 128;
-      const bool need_mask = CAUSAL ? (j == nt - 1) : (kbase + 128 > p.N);
+      const int kbase = j * 128 + 64 * h;
+      const bool need_mask = CAUSAL ? (j == nt - 1) : (j * 128 + 128 > p.N);
       if (need_mask) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
+        for (int c = 0; c < 64; ++c) {
           const int key = kbase + c;
           if (key >= p.N || (CAUSAL && key > qrow)) s[c] = -INFINITY;
         }
       }
-      float bm[8];
+      // Block maxima of the raw scores (sm_scale > 0, so they order like P~).
+      float bm[4];
 #pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        float m0 = s[16 * b];
+      for (int b = 0; b < 4; ++b) {
+        float m0 = max3(s[16 * b], s[16 * b + 1], s[16 * b + 2]);
 #pragma unroll
-        for (int i = 1; i < 16; ++i) m0 = fmaxf(m0, s[16 * b + i]);
-        bm[b] = m0;
+        for (int i = 3; i < 15; i += 2) m0 = max3(m0, s[16 * b + i], s[16 * b + i + 1]);
+        bm[b] = fmaxf(m0, s[16 * b + 15]);
       }
-      float tm = bm[0];
-#pragma unroll
-      for (int b = 1; b < 8; ++b) tm = fmaxf(tm, bm[b]);
+      const float hm = fmaxf(fmaxf(bm[0], bm[1]), fmaxf(bm[2], bm[3]));
+      float* xb = xch + (j & 1) * 256;
+      xb[h * 128 + r] = hm;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_XCH + (j & 1)));
+      if (!__all_sync(0xffffffffu, wait_bar(bar(B_XCH + (j & 1)), (j >> 1) & 1, ctl))) { ok = false; break; }
+      const float tm = fmaxf(hm, xb[(1 - h) * 128 + r]);
+
       const float tmx = tm * xs;
       const float m_new = fmaxf(m_run, tmx);
       const float alpha = ex2_approx(m_run - m_new);
@@ -356,94 +400,67 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float s1 = rfac * (1.0f / 2688.0f);
 
       // Per-16 scales of P2 = P~ / s1 = exp2(S*xs - tmx) * 2688.
-      float inv[8];
-      uint32_t sfw0 = 0, sfw1 = 0;
+      float inv[4];
+      uint32_t sfw = 0;
 #pragma unroll
-      for (int b = 0; b < 8; ++b) {
+      for (int b = 0; b < 4; ++b) {
         const float amax = ex2_approx(fmaf(bm[b], xs, -tmx)) * 2688.0f;
         const uint32_t sbyte = f32_to_e4m3(amax * (1.0f / 6.0f));
         const float sdec = e4m3_to_f32(sbyte);
-        inv[b] = sdec > 0.0f ? 2688.0f / sdec : 0.0f;
-        if (b < 4) sfw0 |= sbyte << (8 * b);
-        else sfw1 |= sbyte << (8 * (b - 4));
+        inv[b] = sdec > 0.0f ? __fdividef(2688.0f, sdec) : 0.0f;
+        sfw |= sbyte << (8 * b);
       }
-      float rowsum = 0.0f;
-      uint32_t pw[16];
+      float2 rs = make_float2(0.0f, 0.0f);
+      uint32_t pw[8];
+      const float2 xs2 = make_float2(xs, xs), nt2 = make_float2(-tmx, -tmx);
 #pragma unroll
-      for (int w = 0; w < 16; ++w) {
-        uint32_t word = 0;
+      for (int w = 0; w < 8; ++w) {
+        const float2 iv = make_float2(inv[w >> 1], inv[w >> 1]);
+        float e[8];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const int k0 = 8 * w + 2 * h;
-          const float e0 = ex2_approx(fmaf(s[k0], xs, -tmx));
-          const float e1 = ex2_approx(fmaf(s[k0 + 1], xs, -tmx));
-          rowsum += e0 + e1;
-          const float iv = inv[k0 / 16];
-          word |= f32x2_to_e2m1(e0 * iv, e1 * iv) << (8 * h);
+        for (int q2 = 0; q2 < 4; ++q2) {
+          const float2 arg = fma2(make_float2(s[8 * w + 2 * q2], s[8 * w + 2 * q2 + 1]), xs2, nt2);
+          const float2 ee = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+          rs = add2(rs, ee);
+          const float2 vv = mul2(ee, iv);
+          e[2 * q2] = vv.x;
+          e[2 * q2 + 1] = vv.y;
         }
-        pw[w] = word;
+        pw[w] = f32x8_to_e2m1(e[0], e[1], e[2], e[3], e[4], e[5], e[6], e[7]);
       }
-      l_run = l_run * alpha + rowsum * rfac;
+      l_half = l_half * alpha + (rs.x + rs.y) * rfac;
       m_run = m_new;
 
       // P^ buffer pb must be free (PV of tile j-2 finished).
-      if (!__all_sync(0xffffffffu, wait_bar(bar(B_PEMPTY + pb), ((j >> 1) & 1) ^ 1, ctl))) break;
+      if (!__all_sync(0xffffffffu, wait_bar(bar(B_PEMPTY + pb), ((j >> 1) & 1) ^ 1, ctl))) { ok = false; break; }
       uint8_t* prow = smem + L::off_p + pb * L::kPBytes + r * 64;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int cs = c ^ ((r >> 1) & 3);
-        *reinterpret_cast<uint4*>(prow + cs * 16) = make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+      for (int c = 0; c < 2; ++c) {
+        const int cs = (2 * h + c) ^ ((r >> 1) & 3);
+        *reinterpret_cast<uint4*>(prow + cs * 16) =
+            make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
       }
-      uint8_t* sfp = smem + L::off_sfp + pb * L::kSfPBytes + (r % 32) * 16 + (r / 32) * 4;
-      *reinterpret_cast<uint32_t*>(sfp) = sfw0;
-      *reinterpret_cast<uint32_t*>(sfp + 512) = sfw1;
+      *reinterpret_cast<uint32_t*>(smem + L::off_sfp + pb * L::kSfPBytes + 512 * h + (r % 32) * 16 + (r / 32) * 4) = sfw;
       fence_proxy_async_smem();
-      float* st = stats + slot * 3 * 128;
-      st[r] = alpha;
-      st[128 + r] = s1;
-      st[256 + r] = l_run;
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar(B_PFULL + pb));
-        mbar_arrive(bar(B_STFULL + slot));
-      }
+      if (lane == 0) mbar_arrive(bar(B_PFULL + pb));
+
+      if (j >= 1 && !correct(j - 1, alpha_prev, s1_prev)) { ok = false; break; }
+      alpha_prev = alpha;
+      s1_prev = s1;
     }
-  } else {
-    // ---------------------------------------------------------- correction ----
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;
-    const int qrow = qt * 128 + r;
-    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    float o[D];
-#pragma unroll
-    for (int d = 0; d < D; ++d) o[d] = 0.0f;
-    float l_fin = 1.0f;
-    bool ok = true;
-    for (int j = 0; j < nt; ++j) {
-      const int slot = j % kStatSlots;
-      if (!__all_sync(0xffffffffu, wait_bar(bar(B_STFULL + slot), (j / kStatSlots) & 1, ctl))) { ok = false; break; }
-      const float* st = stats + slot * 3 * 128;
-      const float alpha = st[r], s1 = st[128 + r];
-      l_fin = st[256 + r];
-      if (!__all_sync(0xffffffffu, wait_bar(bar(B_PVFULL), j & 1, ctl))) { ok = false; break; }
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_base + kColPV + 32 * c, v);
-        tmem_wait_regs(v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[32 * c + i] = fmaf(__uint_as_float(v[i]), s1, o[32 * c + i] * alpha);
-      }
-      tc_fence_before();
+    if (ok) ok = correct(nt - 1, alpha_prev, s1_prev);
+    if (ok) {
+      lsum[h * 128 + r] = l_half;
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_PVEMPTY));
+      if (lane == 0) mbar_arrive(bar(B_LSUM));
+      ok = __all_sync(0xffffffffu, wait_bar(bar(B_LSUM), 0, ctl));
     }
     if (ok && qrow < p.N) {
-      const float il = 1.0f / l_fin;
-      const size_t base = (static_cast<size_t>(bh) * p.N + qrow) * D;
+      const float il = 1.0f / (l_half + lsum[(1 - h) * 128 + r]);
+      const size_t base = (static_cast<size_t>(bh) * p.N + qrow) * D + DH * h;
 #pragma unroll
-      for (int d = 0; d < D; d += 8) {
+      for (int d = 0; d < DH; d += 8) {
         float v8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) v8[i] = o[d + i] * il;

@@ -203,6 +203,56 @@ __device__ __forceinline__ uint32_t f32x2_to_e2m1(float lo, float hi) {
   return r;
 }
 
+// Four pairs of floats -> one 32-bit word of eight E2M1 codes; pair i fills byte i with
+// its first value in the low nibble.
+__device__ __forceinline__ uint32_t f32x8_to_e2m1(float a0, float a1, float b0, float b1, float c0,
+                                                  float c1, float d0, float d1) {
+  uint32_t w;
+  asm("{\n\t.reg .b8 x0, x1, x2, x3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 x0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 x1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 x2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 x3, %8, %7;\n\t"
+      "mov.b32 %0, {x0, x1, x2, x3};\n\t}"
+      : "=r"(w)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1), "f"(d0), "f"(d1));
+  return w;
+}
+
+// Packed two-lane FP32 arithmetic (one instruction for two values).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 p, q, r, s;\n\tmov.b64 p, {%2,%3};\n\tmov.b64 q, {%4,%5};\n\t"
+      "mov.b64 r, {%6,%7};\n\tfma.rn.f32x2 s, p, q, r;\n\tmov.b64 {%0,%1}, s;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 p, q, s;\n\tmov.b64 p, {%2,%3};\n\tmov.b64 q, {%4,%5};\n\t"
+      "mul.rn.f32x2 s, p, q;\n\tmov.b64 {%0,%1}, s;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 p, q, s;\n\tmov.b64 p, {%2,%3};\n\tmov.b64 q, {%4,%5};\n\t"
+      "add.rn.f32x2 s, p, q;\n\tmov.b64 {%0,%1}, s;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
