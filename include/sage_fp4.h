@@ -160,6 +160,12 @@ sage_status_t sage_fp4_qk_scores(const uint8_t* q_fp4, const uint8_t* q_sf, cons
 sage_status_t sage_fp4_get_device_error(uint32_t* word, void* stream);
 
 /*
+ * Text of the last CUDA error that made a call on this host thread return SAGE_ERR_CUDA
+ * (empty if none). Static thread-local storage, valid until the next failing call.
+ */
+const char* sage_fp4_last_cuda_error(void);
+
+/*
  * Bound on every in-kernel wait, in nanoseconds (default 2e9; 0 restores the default).
  * Applies to launches made after the call.
  */

@@ -21,7 +21,8 @@ import torch
 from . import workloads  # noqa: F401  (seeded synthetic inputs)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsage_fp4.so")
+# SAGE_FP4_LIB may point at another build of the same library (A/B comparisons).
+LIB_PATH = os.environ.get("SAGE_FP4_LIB") or os.path.join(_HERE, "libsage_fp4.so")
 
 SAGE_OK, SAGE_ERR_INVALID_ARG, SAGE_ERR_UNSUPPORTED, SAGE_ERR_CUDA, SAGE_ERR_TIMEOUT = range(5)
 SAGE_BF16, SAGE_F16 = 0, 1
@@ -31,13 +32,20 @@ EXPORTED = [
     "sage_fp4_quantize_qkv", "sage_fp4_attn_fwd_quantized", "sage_fp4_workspace_bytes",
     "sage_fp4_attn_fwd_ex", "sage_fp4_attn_fwd", "sage_fp4_qk_scores",
     "sage_fp4_get_device_error", "sage_fp4_set_wait_timeout_ns", "sage_fp4_attn_fwd_noalloc",
+    "sage_fp4_last_cuda_error",
 ]
 
 
 class SageError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {_status_name(status)}")
+        detail = ""
+        if status == SAGE_ERR_CUDA:
+            try:
+                detail = " (" + lib().sage_fp4_last_cuda_error().decode() + ")"
+            except Exception:
+                pass
+        super().__init__(f"{what}: {_status_name(status)}{detail}")
 
 
 class _Sizes(ctypes.Structure):
@@ -73,9 +81,12 @@ def lib():
         L.sage_fp4_qk_scores.argtypes = [u8p, u8p, u8p, u8p, vp, i, i, i, i, f, vp]
         L.sage_fp4_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), vp]
         L.sage_fp4_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+        L.sage_fp4_last_cuda_error.argtypes = []
+        L.sage_fp4_last_cuda_error.restype = ctypes.c_char_p
         L.sage_fp4_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
         for n in EXPORTED[1:]:
-            if n not in ("sage_fp4_quantize_scratch_bytes", "sage_fp4_workspace_bytes"):
+            if n not in ("sage_fp4_quantize_scratch_bytes", "sage_fp4_workspace_bytes",
+                         "sage_fp4_last_cuda_error"):
                 getattr(L, n).restype = i  # sage_status_t
         _lib = L
     return _lib

@@ -394,41 +394,62 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float tm = fmaxf(hm, xb[(1 - h) * 128 + r]);
 
       const float tmx = tm * xs;
-      const float m_new = fmaxf(m_run, tmx);
-      const float alpha = ex2_approx(m_run - m_new);
-      const float rfac = ex2_approx(tmx - m_new);  // rowmax of P~ in this tile
+      // Reference max: it moves only when the tile max exceeds it by more than 8 (log2
+      // units). The reference cancels in O / l, and the P~ quantization below is relative
+      // to the tile max, so this changes rounding only while the O rescale is skipped on
+      // most tiles.
+      const bool move = tmx > m_run + 8.0f;  // always true on the first tile (m_run = -inf)
+      const float m_new = move ? tmx : m_run;
+      const float alpha = move ? ex2_approx(m_run - m_new) : 1.0f;
+      const float rfac = ex2_approx(tmx - m_new);  // rowmax of P~ in this tile (<= 2^8)
       const float s1 = rfac * (1.0f / 2688.0f);
 
-      // Per-16 scales of P2 = P~ / s1 = exp2(S*xs - tmx) * 2688.
-      float inv[4];
-      uint32_t sfw = 0;
+      // Per-16 scales of P2 = P~ / s1 = exp2(S*xs - tmx) * 2688. The division by the
+      // decoded block scale is folded into the exp2 argument: v = exp2(S*xs - nb) = P2 / s.
+      // A block whose scale rounds to zero keeps the plain exp2 (for the row sum) and
+      // gets zero codes.
+      float nb[4], mult[4];
+      uint32_t sfw = 0, zero_blocks = 0;
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
         const float amax = ex2_approx(fmaf(bm[b], xs, -tmx)) * 2688.0f;
         const uint32_t sbyte = f32_to_e4m3(amax * (1.0f / 6.0f));
         const float sdec = e4m3_to_f32(sbyte);
-        inv[b] = sdec > 0.0f ? __fdividef(2688.0f, sdec) : 0.0f;
+        if (sdec > 0.0f) {
+          nb[b] = -(tmx + lg2_approx(sdec) - 11.392317422778761f);  // log2(2688)
+          mult[b] = sdec * (1.0f / 2688.0f);
+        } else {
+          nb[b] = -tmx;
+          mult[b] = 1.0f;
+          zero_blocks |= 1u << b;
+        }
         sfw |= sbyte << (8 * b);
       }
-      float2 rs = make_float2(0.0f, 0.0f);
+      float rsum = 0.0f;
       uint32_t pw[8];
-      const float2 xs2 = make_float2(xs, xs), nt2 = make_float2(-tmx, -tmx);
+      const float2 xs2 = make_float2(xs, xs);
 #pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        const float2 iv = make_float2(inv[w >> 1], inv[w >> 1]);
-        float e[8];
+      for (int b = 0; b < 4; ++b) {
+        const float2 nb2 = make_float2(nb[b], nb[b]);
+        float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
-        for (int q2 = 0; q2 < 4; ++q2) {
-          const float2 arg = fma2(make_float2(s[8 * w + 2 * q2], s[8 * w + 2 * q2 + 1]), xs2, nt2);
-          const float2 ee = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
-          rs = add2(rs, ee);
-          const float2 vv = mul2(ee, iv);
-          e[2 * q2] = vv.x;
-          e[2 * q2 + 1] = vv.y;
+        for (int w = 0; w < 2; ++w) {
+          float e[8];
+#pragma unroll
+          for (int q2 = 0; q2 < 4; ++q2) {
+            const int k0 = 16 * b + 8 * w + 2 * q2;
+            const float2 arg = fma2(make_float2(s[k0], s[k0 + 1]), xs2, nb2);
+            const float2 ee = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+            acc = add2(acc, ee);
+            e[2 * q2] = ee.x;
+            e[2 * q2 + 1] = ee.y;
+          }
+          const uint32_t word = f32x8_to_e2m1(e[0], e[1], e[2], e[3], e[4], e[5], e[6], e[7]);
+          pw[2 * b + w] = (zero_blocks >> b) & 1u ? 0u : word;
         }
-        pw[w] = f32x8_to_e2m1(e[0], e[1], e[2], e[3], e[4], e[5], e[6], e[7]);
+        rsum += (acc.x + acc.y) * mult[b];
       }
-      l_half = l_half * alpha + (rs.x + rs.y) * rfac;
+      l_half = l_half * alpha + rsum * rfac;
       m_run = m_new;
 
       // P^ buffer pb must be free (PV of tile j-2 finished).

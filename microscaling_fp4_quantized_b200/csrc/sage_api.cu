@@ -7,6 +7,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 
@@ -30,7 +31,13 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
 
-sage_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA; }
+thread_local char g_last_error[256] = "";
+
+sage_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SAGE_OK;
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+  return SAGE_ERR_CUDA;
+}
 
 // Address of the device error word on the current device.
 sage_status_t error_word(uint32_t** out) {
@@ -365,6 +372,8 @@ sage_status_t sage_fp4_get_device_error(uint32_t* word, void* stream) {
   *word = host;
   return host == 0 ? SAGE_OK : SAGE_ERR_TIMEOUT;
 }
+
+const char* sage_fp4_last_cuda_error(void) { return g_last_error; }
 
 sage_status_t sage_fp4_set_wait_timeout_ns(uint64_t ns) {
   g_timeout_ns.store(ns == 0 ? kDefaultTimeoutNs : ns);
