@@ -101,6 +101,41 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
 
 
+def _attn_traffic(wl):
+    """DRAM bytes per attention launch from the committed ncu capture, or None when the
+    kernel source has changed since the capture (or no capture exists)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "attn_fp4_fwd_kernel_traffic.json")) as f:
+            rec = json.load(f)
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except Exception:
+        return None, "no capture"
+    if not sha.startswith(rec["source_sha256_prefix"]):
+        return None, "kernel changed since the capture"
+    cap = workloads.by_name(rec["captured_workload"])
+    if cap.name == wl.name:
+        return float(rec["dram_bytes_per_launch"]), f"ncu capture of {cap.name}"
+    # attention traffic is the quantized inputs plus the output: it scales with B*H*N
+    scale = (wl.B * wl.H * wl.N) / (cap.B * cap.H * cap.N)
+    return float(rec["dram_bytes_per_launch"]) * scale, f"ncu capture of {cap.name}, scaled by B*H*N"
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest of the ranks' values (device times are reduced with MAX)."""
+    if dist is None:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(ops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput in TOPS: every rank runs its own copy of the workload."""
+    return world * ops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def cpu_oracle_rate(wl, budget_s: float, q=None, k=None, v=None):
     """Time the CPU oracle (as it stands) on a bounded sample of the workload: one head's
     quantization plus as many query rows as fit the budget; extrapolate to TOPS."""
@@ -216,7 +251,7 @@ def main():
     if sage.device_error() != 0:
         raise RuntimeError("device error word set during warm-up")
 
-    sampler = ClockSampler(local) if rank == 0 or True else None
+    sampler = ClockSampler(local)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
@@ -239,12 +274,9 @@ def main():
     elapsed_ms = t_begin.elapsed_time(t_end)
     attn_ms = [mids[i].elapsed_time(ends[i]) for i in range(args.steps)]
     quant_ms = [starts[i].elapsed_time(mids[i]) for i in range(args.steps)]
-    if dist is not None:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dist, dev)
     ms_per_step = elapsed_ms / args.steps
-    value = world * wl.ops / (ms_per_step * 1e-3) / 1e12
+    value = job_value(wl.ops, world, ms_per_step)
     err = sage.device_error()
 
     # --- end to end through the public API: pinned host inputs -> result on the host ---
@@ -272,13 +304,9 @@ def main():
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1) / e2e_steps
-        if dist is not None:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dist, dev)
         nbytes = q.numel() * q.element_size()
-        e2e = {"value": world * wl.ops / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+        e2e = {"value": job_value(wl.ops, world, e_ms), "unit": UNIT, "ms_per_step": e_ms,
                "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes}
 
     if dist is not None:
@@ -292,9 +320,10 @@ def main():
     fp4_peak = FP4_PER_BF16 * sustained
     attn_avg_ms = statistics.mean(attn_ms)
     achieved = wl.ops / (attn_avg_ms * 1e-3) / 1e12
+    traffic, traffic_src = _attn_traffic(wl)
     roofline = {
         "kernel": "attn_fp4_fwd_kernel", "bound": "tensor", "achieved": achieved, "peak": fp4_peak,
-        "unit": "TFLOP/s", "frac": achieved / fp4_peak, "traffic": None,
+        "unit": "TFLOP/s", "frac": achieved / fp4_peak, "traffic": traffic, "traffic_source": traffic_src,
         "peak_basis": f"{basis} bf16 sustained {sustained} TFLOP/s x {FP4_PER_BF16:g} (nominal FP4:BF16)",
         "frac_of_nominal_9pflops": achieved / FP4_NOMINAL_TFLOPS,
         "attn_ms": attn_avg_ms, "quant_ms": statistics.mean(quant_ms),

@@ -166,6 +166,16 @@ sage_status_t sage_fp4_get_device_error(uint32_t* word, void* stream);
 const char* sage_fp4_last_cuda_error(void);
 
 /*
+ * Test switch for the error path (0 = normal operation, the default). Bit 0: the
+ * attention kernel's copy warp issues no loads, so every wait of the other roles runs
+ * out after the bound set below; the kernel then drains, frees its tensor memory and
+ * returns, and sage_fp4_get_device_error() reports SAGE_ERR_TIMEOUT. Nothing faults and
+ * nothing waits without bound. Applies to launches made after the call; other bits are
+ * rejected with SAGE_ERR_INVALID_ARG.
+ */
+sage_status_t sage_fp4_set_debug_flags(uint32_t flags);
+
+/*
  * Bound on every in-kernel wait, in nanoseconds (default 2e9; 0 restores the default).
  * Applies to launches made after the call.
  */

@@ -32,7 +32,7 @@ EXPORTED = [
     "sage_fp4_quantize_qkv", "sage_fp4_attn_fwd_quantized", "sage_fp4_workspace_bytes",
     "sage_fp4_attn_fwd_ex", "sage_fp4_attn_fwd", "sage_fp4_qk_scores",
     "sage_fp4_get_device_error", "sage_fp4_set_wait_timeout_ns", "sage_fp4_attn_fwd_noalloc",
-    "sage_fp4_last_cuda_error",
+    "sage_fp4_last_cuda_error", "sage_fp4_set_debug_flags",
 ]
 
 
@@ -81,6 +81,7 @@ def lib():
         L.sage_fp4_qk_scores.argtypes = [u8p, u8p, u8p, u8p, vp, i, i, i, i, f, vp]
         L.sage_fp4_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), vp]
         L.sage_fp4_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+        L.sage_fp4_set_debug_flags.argtypes = [ctypes.c_uint32]
         L.sage_fp4_last_cuda_error.argtypes = []
         L.sage_fp4_last_cuda_error.restype = ctypes.c_char_p
         L.sage_fp4_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
@@ -245,6 +246,12 @@ def device_error(device=None) -> int:
 
 def set_wait_timeout_ns(ns: int) -> None:
     _check(lib().sage_fp4_set_wait_timeout_ns(int(ns)), "sage_fp4_set_wait_timeout_ns")
+
+
+def set_debug_flags(flags: int) -> None:
+    """Test switch: bit 0 makes the attention kernel issue no loads, so its bounded waits
+    run out and the device error word reports a timeout (0 restores normal operation)."""
+    _check(lib().sage_fp4_set_debug_flags(int(flags)), "sage_fp4_set_debug_flags")
 
 
 def default_sm_scale(D: int) -> float:

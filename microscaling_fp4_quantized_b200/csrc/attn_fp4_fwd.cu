@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer ----
-    if (lane == 0) {
+    if (lane == 0 && !(p.debug_flags & kDebugNoLoads)) {
       const uint32_t sq = sbase + L::off_q;
       mbar_arrive_expect_tx(bar(B_QFULL), L::kQBytes + L::kSfQKBytes);
       tma_load_2d(sq, &tm_q, 0, bh * p.Np + qt * 128, bar(B_QFULL));

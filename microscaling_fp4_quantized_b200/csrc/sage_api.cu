@@ -20,6 +20,7 @@ __device__ uint32_t g_sage_dev_error;
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
+std::atomic<uint32_t> g_debug_flags{0};
 
 constexpr int kMaxDevices = 64;
 uint32_t* g_err_ptr[kMaxDevices] = {};
@@ -202,6 +203,7 @@ sage_status_t fill_attn_params(const Shape& s, float sm_scale, int causal, sage:
   p->sm_scale_log2 = scale * 1.4426950408889634f;
   p->err = err;
   p->timeout_ns = g_timeout_ns.load();
+  p->debug_flags = g_debug_flags.load();
   return SAGE_OK;
 }
 
@@ -374,6 +376,12 @@ sage_status_t sage_fp4_get_device_error(uint32_t* word, void* stream) {
 }
 
 const char* sage_fp4_last_cuda_error(void) { return g_last_error; }
+
+sage_status_t sage_fp4_set_debug_flags(uint32_t flags) {
+  if (flags & ~1u) return SAGE_ERR_INVALID_ARG;
+  g_debug_flags.store(flags);
+  return SAGE_OK;
+}
 
 sage_status_t sage_fp4_set_wait_timeout_ns(uint64_t ns) {
   g_timeout_ns.store(ns == 0 ? kDefaultTimeoutNs : ns);

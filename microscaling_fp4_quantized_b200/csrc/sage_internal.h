@@ -43,7 +43,10 @@ struct AttnParams {
   float sm_scale_log2;  // sm_scale * log2(e)
   uint32_t* err;        // device error word
   uint64_t timeout_ns;  // bound on every wait
+  uint32_t debug_flags; // kDebugNoLoads: the producer issues no copies (test of the error path)
 };
+
+enum : uint32_t { kDebugNoLoads = 1u };
 
 struct TensorMaps {
   CUtensorMap q, k, v;

@@ -1,0 +1,54 @@
+"""Failure detection without a GPU fault.
+
+The test switch makes the attention kernel issue no loads, so every bounded wait in the
+other roles runs out (50 ms here). The kernel must drain, release its tensor memory and
+return; the host must read a timeout from the device error word; and the same context
+must then run a normal forward that matches the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+from microscaling_fp4_quantized_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sage():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import microscaling_fp4_quantized_b200 as s
+    s.lib()
+    return s
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(sage, oracle_mod):
+    wl = workloads.custom(1, 2, 384, 128, causal=True, seed=61)
+    q, k, v = workloads.make_inputs(wl, device="cuda")
+    assert sage.device_error() == 0
+    sage.set_wait_timeout_ns(50_000_000)
+    sage.set_debug_flags(1)
+    try:
+        sage.attn(q, k, v, causal=True, sm_scale=wl.sm_scale)
+        torch.cuda.synchronize()
+    finally:
+        sage.set_debug_flags(0)
+        sage.set_wait_timeout_ns(0)
+    word = sage.device_error()
+    assert word & 1, f"expected the timeout bit, got {word:#x}"
+    assert sage.device_error() == 0  # reading clears it
+
+    out = sage.attn(q, k, v, causal=True, sm_scale=wl.sm_scale)
+    torch.cuda.synchronize()
+    assert sage.device_error() == 0
+    f = lambda t: t.float().cpu().numpy().reshape(2, wl.N, wl.D)  # noqa: E731
+    em, _ = oracle_mod.attention(f(q), f(k), f(v), True, wl.sm_scale)
+    m = oracle_mod.metrics(f(out), em)
+    assert m["cos"] >= 0.999 and m["max_abs"] <= 1e-2 * float(np.abs(f(v)).max()), m
+
+
+def test_debug_flags_reject_unknown_bits(sage):
+    with pytest.raises(sage.SageError) as e:
+        sage.set_debug_flags(2)
+    assert e.value.status == sage.SAGE_ERR_INVALID_ARG
