@@ -12,8 +12,9 @@ accuracy of the emulated attention against exact attention, which the pages do n
 fix ("parity unpinned" for that comparison; it is reported, not asserted).
 
 Layouts (canonical, row-major; FP4 nibble 2i is the low half of byte i):
-  q_codes, k_codes [BH, N, D/2] uint8; q_sf, k_sf [BH, N, D/16] uint8 (E4M3 bytes)
-  vt_codes [BH, D, Np/2] uint8; vt_sf [BH, D, Np/16] uint8, Np = N rounded up to 16
+  q_codes [B*Hq, Nq, D/2], k_codes [B*Hkv, Nk, D/2] uint8; q_sf, k_sf [..., D/16] uint8
+  (E4M3 bytes); vt_codes [B*Hkv, D, Np/2] uint8; vt_sf [B*Hkv, D, Np/16] uint8, Np = Nk
+  rounded up to 16. Query head h of batch b reads key/value head h / (Hq / Hkv).
 """
 from __future__ import annotations
 
@@ -57,11 +58,14 @@ def _L():
             "so_e4m3_decode": [vp, c_long, vp],
             "so_quant_block16": [vp, c_long, vp, vp],
             "so_kmean": [vp, c_long, c_long, c_long, vp],
-            "so_quantize_qkv": [vp, vp, vp, c_long, c_long, c_long, c_int, vp,
-                                vp, vp, vp, vp, vp, vp, vp],
-            "so_attn_emulated": [vp, vp, vp, vp, vp, vp, c_long, c_long, c_long, c_int,
-                                 c_double, c_long, vp, c_long, vp],
-            "so_attn_exact": [vp, vp, vp, c_long, c_long, c_long, c_int, c_double, vp, c_long, vp],
+            "so_group_amax": [vp, c_long, c_long, c_long, vp, vp],
+            "so_second_level_scale": [vp, c_long, vp],
+            "so_quantize_rows": [vp, c_long, c_long, c_long, vp, vp, vp, vp],
+            "so_quantize_vt": [vp, c_long, c_long, c_long, vp, vp, vp],
+            "so_attn_emulated": [vp, vp, vp, vp, vp, vp, vp, vp, vp, c_long, c_long, c_long,
+                                 c_long, c_long, c_long, c_int, c_double, c_long, vp, c_long, vp],
+            "so_attn_exact": [vp, vp, vp, c_long, c_long, c_long, c_long, c_long, c_long, c_int,
+                              c_double, vp, c_long, vp],
             "so_attn_online": [vp, vp, vp, c_long, c_long, c_long, c_int, c_double, c_long,
                                vp, c_long, vp],
         }
@@ -147,61 +151,130 @@ def kmean(k) -> np.ndarray:
     return out
 
 
-def quantize_qkv(q, k, v, smooth_k: bool = True, kmean_in=None) -> dict:
-    """q, k, v [BH, N, D] (float32 values of the bf16/fp16 inputs) -> canonical arrays."""
-    q, k, v = _f32(q), _f32(k), _f32(v)
-    BH, N, D = q.shape
-    assert k.shape == q.shape == v.shape and D % 16 == 0
+def group_amax(x, mean=None) -> np.ndarray:
+    """x [G, N, D] -> float32 [G]: max |x - mean| (binary32 difference) per group."""
+    x = _f32(x)
+    G, N, D = x.shape
+    m = None if mean is None else _f32(mean).reshape(G, D)
+    out = np.empty(G, np.float32)
+    _L().so_group_amax(_p(x), G, N, D, _p(m) if m is not None else None, _p(out))
+    return out
+
+
+def second_level_scale(amax) -> np.ndarray:
+    """amax -> float32 second-level scales fp32(amax / 2688) (1 where that is 0)."""
+    a = _f32(amax).ravel()
+    out = np.empty(a.shape, np.float32)
+    _L().so_second_level_scale(_p(a), a.size, _p(out))
+    return out.reshape(np.shape(amax))
+
+
+def quantize_rows(x, mean=None, gscale=None):
+    """x [G, N, D] -> (codes [G, N, D/2], sf [G, N, D/16]) along D, after the optional
+    smoothing mean [G, D] and second-level scale [G]."""
+    x = _f32(x)
+    G, N, D = x.shape
+    m = None if mean is None else _f32(mean).reshape(G, D)
+    g = None if gscale is None else _f32(gscale).reshape(G)
+    codes = np.zeros((G, N, D // 2), np.uint8)
+    sf = np.zeros((G, N, D // 16), np.uint8)
+    _L().so_quantize_rows(_p(x), G, N, D, _p(m) if m is not None else None,
+                          _p(g) if g is not None else None, _p(codes), _p(sf))
+    return codes, sf
+
+
+def quantize_vt(v, gscale=None):
+    """v [G, N, D] -> (vt codes [G, D, Np/2], vt sf [G, D, Np/16]), Np = N rounded up to 16."""
+    v = _f32(v)
+    G, N, D = v.shape
     Np = (N + 15) // 16 * 16
-    r = {
-        "q_codes": np.zeros((BH, N, D // 2), np.uint8), "q_sf": np.zeros((BH, N, D // 16), np.uint8),
-        "k_codes": np.zeros((BH, N, D // 2), np.uint8), "k_sf": np.zeros((BH, N, D // 16), np.uint8),
-        "vt_codes": np.zeros((BH, D, Np // 2), np.uint8), "vt_sf": np.zeros((BH, D, Np // 16), np.uint8),
-        "k_mean": np.zeros((BH, D), np.float32), "BH": BH, "N": N, "D": D,
-    }
-    km = None
-    if kmean_in is not None:
-        km = _f32(kmean_in).reshape(BH, D)
-    _L().so_quantize_qkv(_p(q), _p(k), _p(v), BH, N, D, int(bool(smooth_k)),
-                         _p(km) if km is not None else None,
-                         _p(r["q_codes"]), _p(r["q_sf"]), _p(r["k_codes"]), _p(r["k_sf"]),
-                         _p(r["vt_codes"]), _p(r["vt_sf"]), _p(r["k_mean"]))
+    g = None if gscale is None else _f32(gscale).reshape(G)
+    codes = np.zeros((G, D, Np // 2), np.uint8)
+    sf = np.zeros((G, D, Np // 16), np.uint8)
+    _L().so_quantize_vt(_p(v), G, N, D, _p(g) if g is not None else None, _p(codes), _p(sf))
+    return codes, sf
+
+
+GSCALE_MODES = ("none", "tensor", "head")
+
+
+def quantize_qkv(q, k, v, smooth_k: bool = True, kmean_in=None, gscale: str = "none",
+                 amax_in=None, heads=None) -> dict:
+    """Quantize one problem of equal-length sequences.
+
+    q [B*Hq, Nq, D], k and v [B*Hkv, Nk, D] (float32 values of the bf16/fp16 inputs);
+    heads = (B, Hq, Hkv), default (1, q.shape[0], k.shape[0]). K is smoothed by its
+    per-head token mean (kmean_in [B*Hkv, D] supplies it instead). gscale: "none", or a
+    second-level scale per tensor ("tensor") or per head ("head") from the amax of Q,
+    of the smoothed K and of V; amax_in = {"q": [B*Hq], "k": [B*Hkv], "v": [B*Hkv]}
+    supplies those maxima (already reduced for "tensor" mode).
+    """
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    BHq, Nq, D = q.shape
+    BHkv, Nk, Dk = k.shape
+    assert v.shape == k.shape and Dk == D and D % 16 == 0
+    B, Hq, Hkv = heads if heads is not None else (1, BHq, BHkv)
+    assert B * Hq == BHq and B * Hkv == BHkv and Hq % Hkv == 0
+    assert gscale in GSCALE_MODES
+    km = np.zeros((BHkv, D), np.float32)
+    if smooth_k:
+        km = _f32(kmean_in).reshape(BHkv, D) if kmean_in is not None else kmean(k)
+    r = {"B": B, "Hq": Hq, "Hkv": Hkv, "Nq": Nq, "Nk": Nk, "D": D, "k_mean": km,
+         "gq": None, "gk": None, "gv": None, "amax": None}
+    if gscale != "none":
+        if amax_in is not None:
+            am = {n: _f32(amax_in[n]).ravel() for n in ("q", "k", "v")}
+        else:
+            am = {"q": group_amax(q), "k": group_amax(k, km if smooth_k else None), "v": group_amax(v)}
+            if gscale == "tensor":
+                am = {n: np.full(a.shape, a.max(initial=0.0), np.float32) for n, a in am.items()}
+        r["amax"] = am
+        r["gq"], r["gk"], r["gv"] = (second_level_scale(am[n]) for n in ("q", "k", "v"))
+    r["q_codes"], r["q_sf"] = quantize_rows(q, None, r["gq"])
+    r["k_codes"], r["k_sf"] = quantize_rows(k, km if smooth_k else None, r["gk"])
+    r["vt_codes"], r["vt_sf"] = quantize_vt(v, r["gv"])
     return r
 
 
-def _rows(BH: int, N: int, rows) -> np.ndarray:
+def _rows(G: int, N: int, rows) -> np.ndarray:
     if rows is None:
-        bh, i = np.meshgrid(np.arange(BH), np.arange(N), indexing="ij")
-        return np.ascontiguousarray(np.stack([bh.ravel(), i.ravel()], 1).astype(np.int64))
+        g, i = np.meshgrid(np.arange(G), np.arange(N), indexing="ij")
+        return np.ascontiguousarray(np.stack([g.ravel(), i.ravel()], 1).astype(np.int64))
     r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 2))
-    assert (r[:, 0] >= 0).all() and (r[:, 0] < BH).all() and (r[:, 1] >= 0).all() and (r[:, 1] < N).all()
+    assert (r[:, 0] >= 0).all() and (r[:, 0] < G).all() and (r[:, 1] >= 0).all() and (r[:, 1] < N).all()
     return r
 
 
 def attn_emulated(qz: dict, causal: bool, sm_scale: float, Bk: int = 128, rows=None) -> np.ndarray:
-    """Emulated FP4 attention on quantized inputs -> [n_rows, D] binary64 (or [BH, N, D])."""
-    BH, N, D = qz["BH"], qz["N"], qz["D"]
-    r = _rows(BH, N, rows)
+    """Emulated FP4 attention on quantized inputs -> [n_rows, D] binary64 (or
+    [B*Hq, Nq, D] when rows is None). rows are (query head, query index) pairs."""
+    B, Hq, Hkv, Nq, Nk, D = (qz[n] for n in ("B", "Hq", "Hkv", "Nq", "Nk", "D"))
+    r = _rows(B * Hq, Nq, rows)
     out = np.empty((r.shape[0], D), np.float64)
     arrs = [np.ascontiguousarray(qz[n]) for n in ("q_codes", "q_sf", "k_codes", "k_sf", "vt_codes", "vt_sf")]
-    _L().so_attn_emulated(*[_p(a) for a in arrs], BH, N, D, int(bool(causal)), float(sm_scale),
-                          int(Bk), _p(r), r.shape[0], _p(out))
-    return out.reshape(BH, N, D) if rows is None else out
+    gs = [None if qz[n] is None else _f32(qz[n]) for n in ("gq", "gk", "gv")]
+    _L().so_attn_emulated(*[_p(a) for a in arrs], *[_p(g) if g is not None else None for g in gs],
+                          B, Hq, Hkv, Nq, Nk, D, int(bool(causal)), float(sm_scale), int(Bk),
+                          _p(r), r.shape[0], _p(out))
+    return out.reshape(B * Hq, Nq, D) if rows is None else out
 
 
-def attn_exact(q, k, v, causal: bool, sm_scale: float, rows=None) -> np.ndarray:
-    """Two-pass softmax attention in binary64 -> [n_rows, D] (or [BH, N, D])."""
+def attn_exact(q, k, v, causal: bool, sm_scale: float, rows=None, heads=None) -> np.ndarray:
+    """Two-pass softmax attention in binary64 -> [n_rows, D] (or [B*Hq, Nq, D]).
+    q [B*Hq, Nq, D]; k, v [B*Hkv, Nk, D]; heads = (B, Hq, Hkv) as in quantize_qkv."""
     q, k, v = _f32(q), _f32(k), _f32(v)
-    BH, N, D = q.shape
-    r = _rows(BH, N, rows)
+    BHq, Nq, D = q.shape
+    BHkv, Nk, _ = k.shape
+    B, Hq, Hkv = heads if heads is not None else (1, BHq, BHkv)
+    r = _rows(BHq, Nq, rows)
     out = np.empty((r.shape[0], D), np.float64)
-    _L().so_attn_exact(_p(q), _p(k), _p(v), BH, N, D, int(bool(causal)), float(sm_scale),
-                       _p(r), r.shape[0], _p(out))
-    return out.reshape(BH, N, D) if rows is None else out
+    _L().so_attn_exact(_p(q), _p(k), _p(v), B, Hq, Hkv, Nq, Nk, D, int(bool(causal)),
+                       float(sm_scale), _p(r), r.shape[0], _p(out))
+    return out.reshape(BHq, Nq, D) if rows is None else out
 
 
 def attn_online(q, k, v, causal: bool, sm_scale: float, Bk: int = 128, rows=None) -> np.ndarray:
-    """Tiled online-softmax attention in binary64, no quantization."""
+    """Tiled online-softmax attention in binary64, no quantization (Nq == Nk, one head map)."""
     q, k, v = _f32(q), _f32(k), _f32(v)
     BH, N, D = q.shape
     r = _rows(BH, N, rows)
@@ -212,10 +285,100 @@ def attn_online(q, k, v, causal: bool, sm_scale: float, Bk: int = 128, rows=None
 
 
 def attention(q, k, v, causal: bool, sm_scale: float, Bk: int = 128, rows=None,
-              smooth_k: bool = True, kmean_in=None):
+              smooth_k: bool = True, kmean_in=None, gscale: str = "none", heads=None,
+              amax_in=None):
     """Full emulated pipeline: K mean, block quantization, emulated FP4 attention."""
-    qz = quantize_qkv(q, k, v, smooth_k=smooth_k, kmean_in=kmean_in)
+    qz = quantize_qkv(q, k, v, smooth_k=smooth_k, kmean_in=kmean_in, gscale=gscale,
+                      amax_in=amax_in, heads=heads)
     return attn_emulated(qz, causal, sm_scale, Bk=Bk, rows=rows), qz
+
+
+def varlen_amax(q, k, v, cu_q, cu_k, smooth_k: bool = True, kmeans=None) -> dict:
+    """Per-tensor maxima of packed sequences (q [Tq, Hq, D], k, v [Tk, Hkv, D]) for the
+    "tensor" second-level scale: max over every sequence and head, K smoothed by the
+    mean of its own sequence (kmeans[b] [Hkv, D] supplies those)."""
+    a = {"q": 0.0, "k": 0.0, "v": 0.0}
+    for b in range(len(cu_q) - 1):
+        qs = _f32(q[cu_q[b]:cu_q[b + 1]]).transpose(1, 0, 2)
+        ks = _f32(k[cu_k[b]:cu_k[b + 1]]).transpose(1, 0, 2)
+        vs = _f32(v[cu_k[b]:cu_k[b + 1]]).transpose(1, 0, 2)
+        km = None
+        if smooth_k and ks.shape[1] > 0:
+            km = kmeans[b] if kmeans is not None else kmean(ks)
+        if qs.shape[1] > 0:
+            a["q"] = max(a["q"], float(group_amax(qs).max()))
+        if ks.shape[1] > 0:
+            a["k"] = max(a["k"], float(group_amax(ks, km).max()))
+            a["v"] = max(a["v"], float(group_amax(vs).max()))
+    return {n: np.float32(x) for n, x in a.items()}
+
+
+def attention_varlen(q, k, v, cu_q, cu_k, causal: bool, sm_scale: float, Bk: int = 128,
+                     smooth_k: bool = True, gscale: str = "none", kmeans=None, rows=None):
+    """Packed variable-length sequences, each an independent problem.
+
+    q [Tq, Hq, D], k and v [Tk, Hkv, D]; sequence b holds query tokens cu_q[b]..cu_q[b+1]
+    and key tokens cu_k[b]..cu_k[b+1]. Second-level scales: "head" per (sequence, head),
+    "tensor" over all sequences and heads. kmeans[b] [Hkv, D] supplies the K means.
+    rows: (token, head) pairs (None = all). Returns (out [n_rows, D] or [Tq, Hq, D],
+    list of per-sequence quantized dicts).
+    """
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    Tq, Hq, D = q.shape
+    Hkv = k.shape[1]
+    nseq = len(cu_q) - 1
+    am = None
+    if gscale == "tensor":
+        t = varlen_amax(q, k, v, cu_q, cu_k, smooth_k, kmeans)
+    want = np.asarray(rows, np.int64).reshape(-1, 2) if rows is not None else None
+    full = np.zeros((Tq, Hq, D), np.float64)
+    qzs = []
+    for b in range(nseq):
+        Lq, Lk = cu_q[b + 1] - cu_q[b], cu_k[b + 1] - cu_k[b]
+        qs = q[cu_q[b]:cu_q[b + 1]].transpose(1, 0, 2)
+        ks = k[cu_k[b]:cu_k[b + 1]].transpose(1, 0, 2)
+        vs = v[cu_k[b]:cu_k[b + 1]].transpose(1, 0, 2)
+        if Lk == 0 or Lq == 0:
+            qzs.append(None)
+            continue
+        if gscale == "tensor":
+            am = {"q": np.full(Hq, t["q"], np.float32), "k": np.full(Hkv, t["k"], np.float32),
+                  "v": np.full(Hkv, t["v"], np.float32)}
+        sel = None
+        if want is not None:
+            m = (want[:, 0] >= cu_q[b]) & (want[:, 0] < cu_q[b + 1])
+            if not m.any():
+                qzs.append(None)
+                continue
+            sel = np.stack([want[m, 1], want[m, 0] - cu_q[b]], 1)
+        o, qz = attention(qs, ks, vs, causal, sm_scale, Bk=Bk, rows=sel, smooth_k=smooth_k,
+                          kmean_in=None if kmeans is None else kmeans[b], gscale=gscale,
+                          heads=(1, Hq, Hkv), amax_in=am)
+        qzs.append(qz)
+        if sel is None:
+            full[cu_q[b]:cu_q[b + 1]] = o.transpose(1, 0, 2)
+        else:
+            full[sel[:, 1] + cu_q[b], sel[:, 0]] = o
+    if want is not None:
+        return full[want[:, 0], want[:, 1]], qzs
+    return full, qzs
+
+
+def attn_exact_varlen(q, k, v, cu_q, cu_k, causal: bool, sm_scale: float) -> np.ndarray:
+    """Exact attention of packed sequences -> [Tq, Hq, D] binary64."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    Tq, Hq, D = q.shape
+    Hkv = k.shape[1]
+    full = np.zeros((Tq, Hq, D), np.float64)
+    for b in range(len(cu_q) - 1):
+        if cu_q[b + 1] == cu_q[b] or cu_k[b + 1] == cu_k[b]:
+            continue
+        qs = q[cu_q[b]:cu_q[b + 1]].transpose(1, 0, 2)
+        ks = k[cu_k[b]:cu_k[b + 1]].transpose(1, 0, 2)
+        vs = v[cu_k[b]:cu_k[b + 1]].transpose(1, 0, 2)
+        o = attn_exact(qs, ks, vs, causal, sm_scale, heads=(1, Hq, Hkv))
+        full[cu_q[b]:cu_q[b + 1]] = o.transpose(1, 0, 2)
+    return full
 
 
 # ----------------------------------------------------------- error metrics --

@@ -182,61 +182,94 @@ void so_kmean(const float* k, long BH, long N, long D, float* mean) {
   }
 }
 
-// ------------------------------------------------------------ quantize QKV ----
-// Canonical layouts (all row-major, nibble 2i in the low half of byte i):
-//   q_codes, k_codes : [BH, N, D/2]     q_sf, k_sf : [BH, N, D/16]
-//   vt_codes         : [BH, D, Np/2]    vt_sf      : [BH, D, Np/16]
-// where Np = N rounded up to a multiple of 16 (tokens past N count as zeros).
-// K is smoothed as k' = fp32(k - mean) when smooth_k != 0; kmean_in (nullable)
-// supplies the mean instead of computing it; kmean_out (nullable) receives it.
-void so_quantize_qkv(const float* q, const float* k, const float* v, long BH, long N, long D,
-                     int smooth_k, const float* kmean_in, uint8_t* q_codes, uint8_t* q_sf,
-                     uint8_t* k_codes, uint8_t* k_sf, uint8_t* vt_codes, uint8_t* vt_sf,
-                     float* kmean_out) {
-  const long Np = (N + 15) / 16 * 16;
-  std::vector<float> mean(static_cast<size_t>(BH * D), 0.0f);
-  if (smooth_k) {
-    if (kmean_in) std::memcpy(mean.data(), kmean_in, sizeof(float) * BH * D);
-    else so_kmean(k, BH, N, D, mean.data());
+// ------------------------------------------------------ second-level scale ----
+// NVFP4's per-tensor FP32 scale, named (not printed) on the author page ("TetraJet-v2"
+// abstract, "double-block quantization" for NVFP4), read here the way the method scales
+// P~ before its 16-element blocks: a coarse factor maps the largest magnitude of the
+// group onto 448 * 6 (E4M3 max times E2M1 max), the values are divided by it, and the
+// ordinary block rule runs on the quotient.
+//   amax[g] = max |x'| over group g, x' = fp32(x - mean) when a mean is given, else x.
+void so_group_amax(const float* x, long G, long N, long D, const float* mean, float* amax) {
+#pragma omp parallel for schedule(static)
+  for (long g = 0; g < G; ++g) {
+    float a = 0.0f;
+    for (long n = 0; n < N; ++n)
+      for (long d = 0; d < D; ++d) {
+        float v = x[(g * N + n) * D + d];
+        if (mean) v = v - mean[g * D + d];
+        a = std::max(a, std::fabs(v));
+      }
+    amax[g] = a;
   }
-  if (kmean_out) std::memcpy(kmean_out, mean.data(), sizeof(float) * BH * D);
+}
 
+// gscale[i] = fp32(amax[i] / 2688) (binary32 division), or 1 when that is 0.
+void so_second_level_scale(const float* amax, long n, float* gscale) {
+  for (long i = 0; i < n; ++i) {
+    const float g = amax[i] / static_cast<float>(kTwoLevelTarget);
+    gscale[i] = g > 0.0f ? g : 1.0f;
+  }
+}
+
+// ------------------------------------------------------------ quantize rows ----
+// x [G, N, D] quantized along D (the Q and K direction):
+//   x' = fp32(x - mean[g, d])   when mean != NULL (smoothing K),
+//   x'' = fp32(x' / gscale[g])  when gscale != NULL (second-level scale),
+// then the 16-element block rule on x''. Canonical outputs (nibble 2i in the low half
+// of byte i): codes [G, N, D/2], sf [G, N, D/16].
+void so_quantize_rows(const float* x, long G, long N, long D, const float* mean,
+                      const float* gscale, uint8_t* codes, uint8_t* sf) {
   const long nb_d = D / 16;
 #pragma omp parallel for schedule(static)
-  for (long row = 0; row < BH * N; ++row) {
-    const long bh = row / N;
-    float kk[16];
-    uint8_t codes[16];
-    for (long blk = 0; blk < nb_d; ++blk) {
-      const float* qx = q + row * D + blk * 16;
-      quant_block16(qx, 1, 16, codes, &q_sf[row * nb_d + blk]);
-      for (int i = 0; i < 16; ++i) put_nibble(q_codes + row * (D / 2), blk * 16 + i, codes[i]);
-
-      const float* kx = k + row * D + blk * 16;
-      for (int i = 0; i < 16; ++i) kk[i] = kx[i] - mean[bh * D + blk * 16 + i];
-      quant_block16(kk, 1, 16, codes, &k_sf[row * nb_d + blk]);
-      for (int i = 0; i < 16; ++i) put_nibble(k_codes + row * (D / 2), blk * 16 + i, codes[i]);
+  for (long row = 0; row < G * N; ++row) {
+    const long g = row / N;
+    float blk[16];
+    uint8_t c[16];
+    for (long b = 0; b < nb_d; ++b) {
+      for (int i = 0; i < 16; ++i) {
+        float v = x[row * D + b * 16 + i];
+        if (mean) v = v - mean[g * D + b * 16 + i];
+        if (gscale) v = v / gscale[g];
+        blk[i] = v;
+      }
+      quant_block16(blk, 1, 16, c, &sf[row * nb_d + b]);
+      for (int i = 0; i < 16; ++i) put_nibble(codes + row * (D / 2), b * 16 + i, c[i]);
     }
   }
+}
 
+// v [G, N, D] quantized along tokens (the P~V contraction direction) and stored
+// transposed: vt_codes [G, D, Np/2], vt_sf [G, D, Np/16], Np = N rounded up to 16
+// (tokens past N count as zeros). gscale as for so_quantize_rows.
+void so_quantize_vt(const float* v, long G, long N, long D, const float* gscale,
+                    uint8_t* vt_codes, uint8_t* vt_sf) {
+  const long Np = (N + 15) / 16 * 16;
   const long nb_n = Np / 16;
 #pragma omp parallel for schedule(static)
-  for (long bhd = 0; bhd < BH * D; ++bhd) {
-    const long bh = bhd / D, d = bhd % D;
-    uint8_t codes[16];
-    for (long blk = 0; blk < nb_n; ++blk) {
-      const long n0 = blk * 16;
-      const int count = static_cast<int>(std::min<long>(16, N - n0));
-      const float* vx = v + (bh * N + n0) * D + d;
-      quant_block16(vx, D, count, codes, &vt_sf[bhd * nb_n + blk]);
-      for (int i = 0; i < 16; ++i) put_nibble(vt_codes + bhd * (Np / 2), n0 + i, codes[i]);
+  for (long gd = 0; gd < G * D; ++gd) {
+    const long g = gd / D, d = gd % D;
+    float blk[16];
+    uint8_t c[16];
+    for (long b = 0; b < nb_n; ++b) {
+      const long n0 = b * 16;
+      for (int i = 0; i < 16; ++i) {
+        float x = (n0 + i < N) ? v[(g * N + n0 + i) * D + d] : 0.0f;
+        if (gscale) x = x / gscale[g];
+        blk[i] = x;
+      }
+      quant_block16(blk, 1, 16, c, &vt_sf[gd * nb_n + b]);
+      for (int i = 0; i < 16; ++i) put_nibble(vt_codes + gd * (Np / 2), n0 + i, c[i]);
     }
   }
 }
 
 // ------------------------------------------------------ emulated attention ----
-// For each requested row (bh, i): dequantize Q^, K^, V^T exactly in binary64 and walk
-// key tiles of width Bk (the GPU kernel's key-tile width) with the online softmax:
+// One or more sequences of equal lengths: B batches, Hq query heads, Hkv key/value heads
+// (query head h reads key/value head h / (Hq / Hkv)), Nq queries and Nk keys each.
+// Arrays: q codes/sf [B*Hq, Nq, ...]; k codes/sf [B*Hkv, Nk, ...]; vt [B*Hkv, D, ...];
+// gq [B*Hq], gk, gv [B*Hkv] second-level scales (NULL = 1).
+// For each requested row (bhq, i): dequantize exactly in binary64 (code * scale * g)
+// and walk key tiles of width Bk (the GPU kernel's key-tile width) from key 0:
 //   S_j   = sm_scale * sum_d q~_id k~_jd                      (binary64)
 //   m'    = max(m, max_j S_j)   (masked keys excluded)
 //   P~_j  = exp(S_j - m')                                      (masked keys -> 0)
@@ -244,55 +277,62 @@ void so_quantize_qkv(const float* q, const float* k, const float* v, long BH, lo
 //   r     = max_j P~_j ;  s1 = r / (448 * 6)                   (per-row factor)
 //   P2_j  = fp32(P~_j / s1), quantized by the 16-block rule over the tile's keys
 //   O     = O * exp(m - m') + s1 * sum_j p^_j v~_j             (binary64)
-// and finally O / l. Causal masking keeps keys j <= i.
-// rows: n_rows pairs (bh, i); out: [n_rows, D] binary64.
+// and finally O / l. Causal masking keeps keys j <= i + (Nk - Nq) (the last query sees
+// the last key; with Nq == Nk this is j <= i). A row that sees no key gives 0.
+// rows: n_rows pairs (bhq, i); out: [n_rows, D] binary64.
 void so_attn_emulated(const uint8_t* q_codes, const uint8_t* q_sf, const uint8_t* k_codes,
-                      const uint8_t* k_sf, const uint8_t* vt_codes, const uint8_t* vt_sf, long BH,
-                      long N, long D, int causal, double sm_scale, long Bk, const long* rows,
-                      long n_rows, double* out) {
-  const long Np = (N + 15) / 16 * 16;
-  const long nb_d = D / 16, nb_n = Np / 16;
-  // Group rows by head so that K~ and V~ are dequantized once per head.
+                      const uint8_t* k_sf, const uint8_t* vt_codes, const uint8_t* vt_sf,
+                      const float* gq, const float* gk, const float* gv, long B, long Hq,
+                      long Hkv, long Nq, long Nk, long D, int causal, double sm_scale, long Bk,
+                      const long* rows, long n_rows, double* out) {
+  (void)B;
+  const long group = Hq / Hkv;
+  const long Nkp = (Nk + 15) / 16 * 16;
+  const long nb_d = D / 16, nb_n = Nkp / 16;
+  // Group rows by key/value head so that K~ and V~ are dequantized once per head.
+  auto kv_of = [&](long bhq) { return (bhq / Hq) * Hkv + (bhq % Hq) / group; };
   std::vector<long> order(static_cast<size_t>(n_rows));
   for (long r = 0; r < n_rows; ++r) order[r] = r;
   std::stable_sort(order.begin(), order.end(),
-                   [&](long a, long b) { return rows[2 * a] < rows[2 * b]; });
+                   [&](long a, long b) { return kv_of(rows[2 * a]) < kv_of(rows[2 * b]); });
 
-  std::vector<double> kd, vd;  // [N, D] each
+  std::vector<double> kd, vd;  // [Nk, D] each
   long r0 = 0;
   while (r0 < n_rows) {
-    const long bh = rows[2 * order[r0]];
+    const long kv = kv_of(rows[2 * order[r0]]);
     long r1 = r0;
-    while (r1 < n_rows && rows[2 * order[r1]] == bh) ++r1;
+    while (r1 < n_rows && kv_of(rows[2 * order[r1]]) == kv) ++r1;
+    const double g_k = gk ? gk[kv] : 1.0, g_v = gv ? gv[kv] : 1.0;
 
-    kd.assign(static_cast<size_t>(N * D), 0.0);
-    vd.assign(static_cast<size_t>(N * D), 0.0);
+    kd.assign(static_cast<size_t>(Nk * D), 0.0);
+    vd.assign(static_cast<size_t>(Nk * D), 0.0);
 #pragma omp parallel for schedule(static)
-    for (long n = 0; n < N; ++n) {
-      const uint8_t* kr = k_codes + (bh * N + n) * (D / 2);
+    for (long n = 0; n < Nk; ++n) {
+      const uint8_t* kr = k_codes + (kv * Nk + n) * (D / 2);
       for (long d = 0; d < D; ++d) {
-        const double s = e4m3_value(k_sf[(bh * N + n) * nb_d + d / 16]);
-        kd[n * D + d] = e2m1_value(get_nibble(kr, d)) * s;
-        const uint8_t* vr = vt_codes + (bh * D + d) * (Np / 2);
-        const double sv = e4m3_value(vt_sf[(bh * D + d) * nb_n + n / 16]);
-        vd[n * D + d] = e2m1_value(get_nibble(vr, n)) * sv;
+        const double s = e4m3_value(k_sf[(kv * Nk + n) * nb_d + d / 16]);
+        kd[n * D + d] = e2m1_value(get_nibble(kr, d)) * s * g_k;
+        const uint8_t* vr = vt_codes + (kv * D + d) * (Nkp / 2);
+        const double sv = e4m3_value(vt_sf[(kv * D + d) * nb_n + n / 16]);
+        vd[n * D + d] = e2m1_value(get_nibble(vr, n)) * sv * g_v;
       }
     }
 
 #pragma omp parallel for schedule(dynamic, 1)
     for (long rr = r0; rr < r1; ++rr) {
       const long ridx = order[rr];
-      const long i = rows[2 * ridx + 1];
+      const long bhq = rows[2 * ridx], i = rows[2 * ridx + 1];
+      const double g_q = gq ? gq[bhq] : 1.0;
       std::vector<double> qd(static_cast<size_t>(D)), O(static_cast<size_t>(D), 0.0);
       std::vector<double> S(static_cast<size_t>(Bk)), P(static_cast<size_t>(Bk));
       std::vector<float> P2(static_cast<size_t>(Bk + 16));
       std::vector<double> phat(static_cast<size_t>(Bk + 16));
-      const uint8_t* qr = q_codes + (bh * N + i) * (D / 2);
+      const uint8_t* qr = q_codes + (bhq * Nq + i) * (D / 2);
       for (long d = 0; d < D; ++d)
-        qd[d] = e2m1_value(get_nibble(qr, d)) * e4m3_value(q_sf[(bh * N + i) * nb_d + d / 16]);
+        qd[d] = e2m1_value(get_nibble(qr, d)) * e4m3_value(q_sf[(bhq * Nq + i) * nb_d + d / 16]) * g_q;
 
       double m = -std::numeric_limits<double>::infinity(), l = 0.0;
-      const long last_key = causal ? std::min(i, N - 1) : N - 1;
+      const long last_key = causal ? std::min(i + (Nk - Nq), Nk - 1) : Nk - 1;
       for (long j0 = 0; j0 <= last_key; j0 += Bk) {
         const long j1 = std::min(j0 + Bk, last_key + 1);  // exclusive; keys past it are masked
         double tmax = -std::numeric_limits<double>::infinity();
@@ -329,7 +369,7 @@ void so_attn_emulated(const uint8_t* q_codes, const uint8_t* q_sf, const uint8_t
         }
         m = m_new;
       }
-      for (long d = 0; d < D; ++d) out[ridx * D + d] = O[d] / l;
+      for (long d = 0; d < D; ++d) out[ridx * D + d] = l > 0.0 ? O[d] / l : 0.0;
     }
     r0 = r1;
   }
@@ -337,19 +377,25 @@ void so_attn_emulated(const uint8_t* q_codes, const uint8_t* q_sf, const uint8_t
 
 // --------------------------------------------------- unquantized attention ----
 // Plain two-pass softmax attention in binary64 on the fp32 inputs (the definition):
-//   O_i = sum_j exp(S_ij - max_j S_ij) v_j / sum_j exp(S_ij - max_j S_ij).
-void so_attn_exact(const float* q, const float* k, const float* v, long BH, long N, long D,
-                   int causal, double sm_scale, const long* rows, long n_rows, double* out) {
+//   O_i = sum_j exp(S_ij - max_j S_ij) v_j / sum_j exp(S_ij - max_j S_ij),
+// with the head map and causal rule of so_attn_emulated (keys j <= i + Nk - Nq; a row
+// with no visible key gives 0). q [B*Hq, Nq, D]; k, v [B*Hkv, Nk, D].
+void so_attn_exact(const float* q, const float* k, const float* v, long B, long Hq, long Hkv,
+                   long Nq, long Nk, long D, int causal, double sm_scale, const long* rows,
+                   long n_rows, double* out) {
+  (void)B;
+  const long group = Hq / Hkv;
 #pragma omp parallel for schedule(dynamic, 1)
   for (long r = 0; r < n_rows; ++r) {
-    const long bh = rows[2 * r], i = rows[2 * r + 1];
-    const long nk = causal ? std::min(i + 1, N) : N;
+    const long bhq = rows[2 * r], i = rows[2 * r + 1];
+    const long kv = (bhq / Hq) * Hkv + (bhq % Hq) / group;
+    const long nk = causal ? std::max(0L, std::min(i + 1 + (Nk - Nq), Nk)) : Nk;
     std::vector<double> S(static_cast<size_t>(nk));
     double mx = -std::numeric_limits<double>::infinity();
     for (long j = 0; j < nk; ++j) {
       double acc = 0.0;
       for (long d = 0; d < D; ++d)
-        acc += static_cast<double>(q[(bh * N + i) * D + d]) * static_cast<double>(k[(bh * N + j) * D + d]);
+        acc += static_cast<double>(q[(bhq * Nq + i) * D + d]) * static_cast<double>(k[(kv * Nk + j) * D + d]);
       S[j] = sm_scale * acc;
       mx = std::max(mx, S[j]);
     }
@@ -360,8 +406,8 @@ void so_attn_exact(const float* q, const float* k, const float* v, long BH, long
     }
     for (long d = 0; d < D; ++d) {
       double acc = 0.0;
-      for (long j = 0; j < nk; ++j) acc += S[j] * static_cast<double>(v[(bh * N + j) * D + d]);
-      out[r * D + d] = acc / l;
+      for (long j = 0; j < nk; ++j) acc += S[j] * static_cast<double>(v[(kv * Nk + j) * D + d]);
+      out[r * D + d] = nk > 0 ? acc / l : 0.0;
     }
   }
 }
