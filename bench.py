@@ -203,6 +203,53 @@ def run_reference(args, wl):
     return 0
 
 
+# Kernels per step: K statistics, K mean, quantization, attention.
+LAUNCHES_PER_STEP = 4
+
+
+def time_general(sage, gw, dev, stream, warmup, steps, inputs=None):
+    """Whole forward of a general workload through sageattn / sageattn_varlen with a
+    preallocated workspace: CUDA events on the launching stream, median per step."""
+    if inputs is None:
+        x = workloads.make_general_inputs(gw, dev)
+    else:
+        x = {"q": inputs[0], "k": inputs[1], "v": inputs[2]}
+    out = torch.empty(x["q"].shape, dtype=x["q"].dtype, device=dev)
+    if gw.packed:
+        pr = sage.sageattn_varlen_problem(x["q"], x["k"], x["v"], out, x["cu_seqlens_q"],
+                                          x["cu_seqlens_k"], max(gw.lens_q), max(gw.lens_k),
+                                          gw.causal, None, True, gw.gscale)
+    else:
+        pr = sage.sageattn_problem(x["q"], x["k"], x["v"], out, gw.layout, gw.causal, None, True,
+                                   gw.gscale)
+    ws = torch.empty(sage.problem_sizes(pr)["workspace"], dtype=torch.uint8, device=dev)
+
+    def run():
+        if gw.packed:
+            sage.sageattn_varlen(x["q"], x["k"], x["v"], x["cu_seqlens_q"], x["cu_seqlens_k"],
+                                 max(gw.lens_q), max(gw.lens_k), is_causal=gw.causal,
+                                 gscale=gw.gscale, out=out, workspace=ws)
+        else:
+            sage.sageattn(x["q"], x["k"], x["v"], tensor_layout=gw.layout, is_causal=gw.causal,
+                          gscale=gw.gscale, out=out, workspace=ws)
+
+    for _ in range(max(warmup, 3)):
+        run()
+    torch.cuda.synchronize()
+    if sage.device_error() != 0:
+        raise RuntimeError(f"device error word set running {gw.name}")
+    ts = []
+    for _ in range(steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run()
+        e1.record(stream)
+        ts.append((e0, e1))
+    torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(b) for a, b in ts)
+    return {"ms_per_step": ms, "value": gw.ops / (ms * 1e-3) / 1e12, "unit": UNIT}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -213,6 +260,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--variants", action="store_true",
+                    help="also time the general-problem paths (second-level scales, packed "
+                         "grouped-query batch) and report them under 'variants'")
     args = ap.parse_args()
     wl = workloads.by_name(args.workload)
     if args.impl == "reference":
@@ -309,6 +359,18 @@ def main():
         e2e = {"value": job_value(wl.ops, world, e_ms), "unit": UNIT, "ms_per_step": e_ms,
                "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes}
 
+    variants = None
+    if args.variants:
+        variants = {}
+        for g in ("tensor", "head"):
+            gw = workloads.general(f"{wl.name}_gscale_{g}", wl.H, wl.H, wl.D, (wl.N,) * wl.B,
+                                   causal=wl.causal, packed=False, seed=wl.seed, gscale=g)
+            variants[gw.name] = time_general(sage, gw, dev, stream, args.warmup, min(args.steps, 20),
+                                             inputs=(qd, kd, vd))
+        gw = workloads.LLM_VARLEN_GQA
+        variants[gw.name] = time_general(sage, gw, dev, stream, args.warmup, min(args.steps, 20))
+        variants[gw.name]["config"] = gw.describe()
+
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -340,9 +402,11 @@ def main():
         "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp4_e2m1", "data": "synthetic",
         "config": cfg, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": 3 * args.steps, "clocks": clocks, "device_error_word": err,
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clocks, "device_error_word": err,
         "pct_of_fp4_peak": 100.0 * value / world / fp4_peak,
     }
+    if variants is not None:
+        line["variants"] = variants
     print(json.dumps(line), flush=True)
     return 0
 

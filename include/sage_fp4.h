@@ -17,13 +17,24 @@
  *   4. P~ quantized with two-level scaling: a per-row factor s1 = rowmax(P~)/(448*6)
  *      per key tile, then the same 16-element E4M3/E2M1 rule; P^ V^ as a second
  *      block-scaled FP4 contraction, accumulated in FP32.
+ *   5. Optional (sage_fp4_problem_t.gscale): a second-level FP32 scale per tensor or per
+ *      (sequence, head) for Q, K' and V, NVFP4's per-tensor factor (named on the author
+ *      page, "TetraJet-v2" abstract: double-block quantization for NVFP4), applied the
+ *      way step 4 scales P~: g = amax / (448*6), the 16-element rule runs on x / g, and
+ *      g is folded back into the scores (Q, K) and the output (V).
  *
  * Conventions for every entry point
  *   - Tensors are device pointers unless stated; the caller owns all memory. The
  *     library keeps no per-call state and never frees caller memory.
- *   - Q, K, V, O: [B, H, N, D] contiguous, element type bf16 or fp16 (sage_dtype_t).
+ *   - Dense entry points: Q, K, V, O are [B, H, N, D] contiguous, element type bf16 or
+ *     fp16 (sage_dtype_t). sage_fp4_problem_t describes the general case: any token /
+ *     head / batch strides, packed variable-length sequences, key/value heads shared by
+ *     groups of query heads, and query and key lengths that differ.
  *   - D must be 64 or 128; B, H, N >= 0 (any zero gives an empty problem: SAGE_OK,
  *     nothing launched); N need not be a multiple of anything.
+ *   - Causal masking keeps key j for query i when j <= i + (len_k - len_q): the last
+ *     query sees the last key (with len_q == len_k, j <= i). A query that sees no key
+ *     (or a sequence with no keys) gets an output row of zeros.
  *   - All pointers must be 16-byte aligned.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call is
  *     asynchronous on it; argument errors are returned before anything is launched.
@@ -33,21 +44,28 @@
  *     a device error word, the kernel drains its own copies, frees its tensor memory
  *     and returns; sage_fp4_get_device_error() reports it (SAGE_ERR_TIMEOUT).
  *
- * Quantized layouts (Np = N rounded up to a multiple of 128; rows/tokens >= N are 0):
- *   q_fp4, k_fp4 : [B*H, Np, D/2] bytes. Byte j of row n holds elements 2j (low nibble)
- *                  and 2j+1 (high nibble) of that row. E2M1 code = sign<<3 | magnitude.
- *   vt_fp4       : [B*H, D, Np/2] bytes: V transposed; byte j of row d holds tokens 2j
- *                  (low nibble) and 2j+1 (high nibble).
- *   q_sf, k_sf   : [B*H, Np/128, D/64, 512] bytes, the tensor-core scale-factor tiling.
- *                  The scale of (bh, token n, channels 16c..16c+15) is at
- *                    ((bh*(Np/128) + n/128) * (D/64) + (16c)/64) * 512
- *                    + (n%32)*16 + ((n%128)/32)*4 + c%4
- *   vt_sf        : [B*H, Np/128, 2, 512] bytes. The scale of (bh, channel d, tokens
- *                  16t..16t+15) is at
- *                    ((bh*(Np/128) + (16t)/128) * 2 + ((16t)%128)/64) * 512
- *                    + (d%32)*16 + (d/32)*4 + t%4
+ * Quantized layouts. Every sequence is padded to a multiple of 128 tokens (padding
+ * tokens quantize as zeros). For the dense [B, H, N, D] entry points let Np = N rounded
+ * up to 128; the padded row of (batch b, head h, token n) is then (b*H + h)*Np + n.
+ * In general (sage_fp4_problem_t) the padded row of query (sequence b, head h, token n)
+ * is  Hq * P_b + h * round128(len_q(b)) + n,  where P_b is the sum of round128(len_q)
+ * over the sequences before b (b * round128(Nq) for dense problems); keys use Hkv,
+ * len_k and their own P_b. A "tile" is 128 consecutive padded rows: tile t = row / 128.
+ *   q_fp4, k_fp4 : [rows, D/2] bytes. Byte j of a row holds elements 2j (low nibble)
+ *                  and 2j+1 (high nibble). E2M1 code = sign<<3 | magnitude.
+ *   vt_fp4       : [key tiles, D, 64] bytes: V transposed per key tile; byte j of row d
+ *                  of tile t holds tokens 128t + 2j (low nibble) and 128t + 2j + 1.
+ *   q_sf, k_sf   : [tiles, D/64, 512] bytes, the tensor-core scale-factor tiling. The
+ *                  scale of (row r, channels 16c..16c+15) is at
+ *                    ((r/128) * (D/64) + (16c)/64) * 512 + (r%32)*16 + ((r%128)/32)*4 + c%4
+ *   vt_sf        : [key tiles, 2, 512] bytes. The scale of (channel d, tokens
+ *                  16u..16u+15 of tile t, u < 8) is at
+ *                    (t * 2 + u/4) * 512 + (d%32)*16 + (d/32)*4 + u%4
  *                  (for D = 64 the bytes with d/32 >= 2 are 0).
- *   k_mean       : [B*H, D] float32: fp32(sum_n K[bh, n, d] in binary64 / N).
+ *   k_mean       : [B*Hkv, D] float32: fp32(sum_n K[b, h, n, d] in binary64 / len_k).
+ *   amax         : [3, B*Hq] float32, second-level maxima of Q, K - mean and V (element
+ *                  b*Hq + h for Q and b*Hkv + h for K and V; element 0 of each in the
+ *                  per-tensor mode); the scale is fp32(amax / 2688), or 1 if that is 0.
  */
 #ifndef SAGE_FP4_H
 #define SAGE_FP4_H
@@ -61,7 +79,8 @@ extern "C" {
 
 typedef enum {
   SAGE_OK = 0,
-  SAGE_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, short workspace */
+  SAGE_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, short workspace,
+                               (from sage_fp4_get_device_error) a bad sequence table */
   SAGE_ERR_UNSUPPORTED = 2, /* D not in {64, 128}, or a size beyond the 32-bit indexing limits */
   SAGE_ERR_CUDA = 3,        /* a CUDA runtime/driver call or launch failed */
   SAGE_ERR_TIMEOUT = 4      /* a bounded wait inside a kernel ran out (see above) */
@@ -72,13 +91,95 @@ typedef enum { SAGE_BF16 = 0, SAGE_F16 = 1 } sage_dtype_t;
 /* Human-readable name of a status code (static storage). */
 const char* sage_status_string(sage_status_t status);
 
+/* ---------------------------------------------------------------- general problem ---- */
+
+typedef enum {
+  SAGE_GSCALE_NONE = 0,   /* one level: the 16-element E4M3 scales alone (the method as stated) */
+  SAGE_GSCALE_TENSOR = 1, /* plus one FP32 scale per tensor (Q, K - mean, V): NVFP4's shape */
+  SAGE_GSCALE_HEAD = 2    /* plus one FP32 scale per (sequence, head) of each tensor */
+} sage_gscale_t;
+
+/*
+ * One attention problem. Element (sequence b, head h, token n, channel d) of Q is at
+ *   q + (b*q_stride[0] + h*q_stride[1] + (t0 + n)*q_stride[2] + d) elements,
+ * t0 = 0 for dense problems and cu_seqlens_q[b] for packed ones (whose batch stride is
+ * ignored); K, V and O likewise (K and V with cu_seqlens_k). Channels are contiguous;
+ * every stride must be a non-negative multiple of 8 elements (16 bytes). The library
+ * cannot check that the strides stay inside the caller's allocations.
+ */
+typedef struct {
+  int B;                        /* sequences */
+  int Hq, Hkv;                  /* query heads; key/value heads (Hq % Hkv == 0) */
+  int D;                        /* head dimension: 64 or 128 */
+  int Nq, Nk;                   /* dense: tokens per sequence; packed: the longest sequence */
+  const int32_t* cu_seqlens_q;  /* packed: device [B+1] token offsets into q and out, else NULL */
+  const int32_t* cu_seqlens_k;  /* packed: device [B+1] token offsets into k and v, else NULL */
+  int total_q, total_k;         /* packed: tokens in the packed tensors (= cu_seqlens[B]) */
+  int64_t q_stride[3];          /* elements between consecutive (sequence, head, token) */
+  int64_t k_stride[3];
+  int64_t v_stride[3];
+  int64_t o_stride[3];
+  sage_dtype_t dtype;           /* of q, k, v and out */
+  int causal;
+  float sm_scale;               /* <= 0: 1/sqrt(D) */
+  int smooth_k;                 /* subtract the per-(sequence, head) channel mean of K */
+  sage_gscale_t gscale;
+} sage_fp4_problem_t;
+
+/* The quantized tensors of a problem (layouts above); device pointers, 16-byte aligned. */
+typedef struct {
+  uint8_t *q_fp4, *q_sf, *k_fp4, *k_sf, *vt_fp4, *vt_sf;
+  float* k_mean;                /* required by sage_fp4_quantize */
+  float* amax;                  /* required when gscale != SAGE_GSCALE_NONE */
+  int32_t* seq;                 /* packed problems: the padded offsets of every sequence,
+                                   [2, B+1] int32 plus a validity word; else unused */
+} sage_fp4_quantized_t;
+
+/* Byte sizes for a problem (all 0 for an empty problem). For packed problems the
+ * quantized sizes are upper bounds computed from B, Nq, Nk, total_q and total_k. */
+typedef struct {
+  size_t q_fp4, q_sf, k_fp4, k_sf, vt_fp4, vt_sf, k_mean, amax, seq;
+  size_t scratch;    /* scratch of sage_fp4_quantize */
+  size_t workspace;  /* workspace of sage_fp4_attn: the above, each 256-byte aligned */
+} sage_fp4_problem_sizes_t;
+
+sage_status_t sage_fp4_problem_sizes(const sage_fp4_problem_t* problem, sage_fp4_problem_sizes_t* sizes);
+
+/*
+ * Steps 1-2 (and 5) for a general problem: K mean, second-level maxima, quantization of
+ * Q, K - mean and V^T into the buffers of `qz`. Packed problems first check the sequence
+ * table on the device (cu_seqlens start at 0, do not decrease, end at total_q / total_k,
+ * no sequence longer than Nq / Nk); a table that fails sets the device error word
+ * (sage_fp4_get_device_error returns SAGE_ERR_INVALID_ARG) and every later kernel of
+ * the call leaves its outputs untouched. scratch: at least sizes.scratch bytes.
+ */
+sage_status_t sage_fp4_quantize(const sage_fp4_problem_t* problem, const void* q, const void* k,
+                                const void* v, const sage_fp4_quantized_t* qz, void* scratch,
+                                size_t scratch_bytes, void* stream);
+
+/* Steps 3-4 on the output of sage_fp4_quantize for the same problem (k_mean unused). */
+sage_status_t sage_fp4_attn_quantized(const sage_fp4_problem_t* problem, const sage_fp4_quantized_t* qz,
+                                      void* out, void* stream);
+
+/*
+ * The whole forward of a general problem with a caller-owned workspace of at least
+ * sizes.workspace bytes (256-byte aligned). Dense problems without a second-level scale
+ * launch 4 kernels (K statistics, K mean, quantization, attention); packed problems add
+ * the sequence-table kernel.
+ */
+sage_status_t sage_fp4_attn(const sage_fp4_problem_t* problem, const void* q, const void* k,
+                            const void* v, void* out, void* workspace, size_t ws_bytes, void* stream);
+
+/* -------------------------------------------------- dense [B, H, N, D] problems ---- */
+
 /* Byte sizes of the quantized tensors for a problem (0 for an empty problem). */
 typedef struct {
   size_t q_fp4, q_sf, k_fp4, k_sf, vt_fp4, vt_sf, k_mean;
 } sage_fp4_sizes_t;
 sage_status_t sage_fp4_quantized_sizes(int B, int H, int N, int D, sage_fp4_sizes_t* sizes);
 
-/* Scratch bytes sage_fp4_quantize_qkv needs (binary64 partial sums for the K mean). */
+/* Scratch bytes sage_fp4_quantize_qkv needs (binary64 partial sums for the K mean, and
+ * room for the mean itself when k_mean is NULL). */
 size_t sage_fp4_quantize_scratch_bytes(int B, int H, int N, int D);
 
 /*
@@ -108,7 +209,7 @@ size_t sage_fp4_workspace_bytes(int B, int H, int N, int D);
 
 /*
  * The whole forward (steps 1-4) with a caller-owned workspace of at least
- * sage_fp4_workspace_bytes() bytes (256-byte aligned). Three kernel launches.
+ * sage_fp4_workspace_bytes() bytes (256-byte aligned). Four kernel launches.
  */
 sage_status_t sage_fp4_attn_fwd_ex(const void* q, const void* k, const void* v, void* out,
                                    sage_dtype_t dtype, int B, int H, int N, int D, int causal,

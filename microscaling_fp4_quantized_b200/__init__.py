@@ -8,6 +8,8 @@ no CPU fallback: if the library cannot be loaded, every call raises.
 
     import microscaling_fp4_quantized_b200 as sage
     out = sage.attn(q, k, v, causal=False)          # q, k, v: [B, H, N, D] bf16/fp16 CUDA
+    out = sage.sageattn(q, k, v, tensor_layout="NHD", is_causal=True)   # strided, GQA
+    out = sage.sageattn_varlen(q, k, v, cu_q, cu_k, max_q, max_k)      # packed sequences
 """
 from __future__ import annotations
 
@@ -26,13 +28,15 @@ LIB_PATH = os.environ.get("SAGE_FP4_LIB") or os.path.join(_HERE, "libsage_fp4.so
 
 SAGE_OK, SAGE_ERR_INVALID_ARG, SAGE_ERR_UNSUPPORTED, SAGE_ERR_CUDA, SAGE_ERR_TIMEOUT = range(5)
 SAGE_BF16, SAGE_F16 = 0, 1
+GSCALE = {"none": 0, "tensor": 1, "head": 2}
 
 EXPORTED = [
     "sage_status_string", "sage_fp4_quantized_sizes", "sage_fp4_quantize_scratch_bytes",
     "sage_fp4_quantize_qkv", "sage_fp4_attn_fwd_quantized", "sage_fp4_workspace_bytes",
     "sage_fp4_attn_fwd_ex", "sage_fp4_attn_fwd", "sage_fp4_qk_scores",
     "sage_fp4_get_device_error", "sage_fp4_set_wait_timeout_ns", "sage_fp4_attn_fwd_noalloc",
-    "sage_fp4_last_cuda_error", "sage_fp4_set_debug_flags",
+    "sage_fp4_last_cuda_error", "sage_fp4_set_debug_flags", "sage_fp4_problem_sizes",
+    "sage_fp4_quantize", "sage_fp4_attn_quantized", "sage_fp4_attn",
 ]
 
 
@@ -50,6 +54,28 @@ class SageError(RuntimeError):
 
 class _Sizes(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in ("q_fp4", "q_sf", "k_fp4", "k_sf", "vt_fp4", "vt_sf", "k_mean")]
+
+
+class _Problem(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("D", ctypes.c_int),
+                ("Nq", ctypes.c_int), ("Nk", ctypes.c_int),
+                ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_k", ctypes.c_void_p),
+                ("total_q", ctypes.c_int), ("total_k", ctypes.c_int),
+                ("q_stride", ctypes.c_int64 * 3), ("k_stride", ctypes.c_int64 * 3),
+                ("v_stride", ctypes.c_int64 * 3), ("o_stride", ctypes.c_int64 * 3),
+                ("dtype", ctypes.c_int), ("causal", ctypes.c_int), ("sm_scale", ctypes.c_float),
+                ("smooth_k", ctypes.c_int), ("gscale", ctypes.c_int)]
+
+
+_QZ_FIELDS = ("q_fp4", "q_sf", "k_fp4", "k_sf", "vt_fp4", "vt_sf", "k_mean", "amax", "seq")
+
+
+class _Quantized(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _QZ_FIELDS]
+
+
+class _ProblemSizes(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in _QZ_FIELDS + ("scratch", "workspace")]
 
 
 _lib = None
@@ -85,6 +111,11 @@ def lib():
         L.sage_fp4_last_cuda_error.argtypes = []
         L.sage_fp4_last_cuda_error.restype = ctypes.c_char_p
         L.sage_fp4_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
+        pp = ctypes.POINTER(_Problem)
+        L.sage_fp4_problem_sizes.argtypes = [pp, ctypes.POINTER(_ProblemSizes)]
+        L.sage_fp4_quantize.argtypes = [pp, vp, vp, vp, ctypes.POINTER(_Quantized), vp, sz, vp]
+        L.sage_fp4_attn_quantized.argtypes = [pp, ctypes.POINTER(_Quantized), vp, vp]
+        L.sage_fp4_attn.argtypes = [pp, vp, vp, vp, vp, vp, sz, vp]
         for n in EXPORTED[1:]:
             if n not in ("sage_fp4_quantize_scratch_bytes", "sage_fp4_workspace_bytes",
                          "sage_fp4_last_cuda_error"):
@@ -235,11 +266,15 @@ def qk_scores(qz: dict, sm_scale: Optional[float] = None) -> torch.Tensor:
     return s
 
 
+DEV_ERR_TIMEOUT, DEV_ERR_SEQLENS = 1, 2
+
+
 def device_error(device=None) -> int:
-    """Read and clear the device error word (synchronizes the current stream)."""
+    """Read and clear the device error word (synchronizes the current stream): bit 0 a
+    bounded wait ran out, bit 1 a packed problem's sequence table failed its check."""
     w = ctypes.c_uint32(0)
     st = lib().sage_fp4_get_device_error(ctypes.byref(w), _stream(device))
-    if st not in (SAGE_OK, SAGE_ERR_TIMEOUT):
+    if st not in (SAGE_OK, SAGE_ERR_TIMEOUT, SAGE_ERR_INVALID_ARG):
         raise SageError(st, "sage_fp4_get_device_error")
     return int(w.value)
 
@@ -288,3 +323,168 @@ class Plan:
             _ptr(b["vt_sf"]), _ptr(out), _dtype_code(out.dtype), self.B, self.H, self.N, self.D,
             int(bool(causal)), float(sm_scale or 0.0), _stream(self.device)),
             "sage_fp4_attn_fwd_quantized")
+
+
+# ------------------------------------------------------------------ general problems --
+
+def _strides3(t: torch.Tensor, dims) -> tuple:
+    if t.stride(-1) != 1:
+        raise ValueError("the channel (last) dimension must be contiguous")
+    return tuple(int(t.stride(d)) for d in dims)
+
+
+def make_problem(*, B: int, Hq: int, Hkv: int, D: int, Nq: int, Nk: int, dtype: torch.dtype,
+                 q_stride, k_stride, v_stride, o_stride, causal: bool = False,
+                 sm_scale: Optional[float] = None, smooth_k: bool = True, gscale: str = "none",
+                 cu_seqlens_q: Optional[torch.Tensor] = None,
+                 cu_seqlens_k: Optional[torch.Tensor] = None, total_q: int = 0,
+                 total_k: int = 0) -> _Problem:
+    """The C problem descriptor (strides in elements of (sequence, head, token))."""
+    if gscale not in GSCALE:
+        raise ValueError(f"gscale must be one of {tuple(GSCALE)}")
+    pr = _Problem()
+    pr.B, pr.Hq, pr.Hkv, pr.D, pr.Nq, pr.Nk = B, Hq, Hkv, D, Nq, Nk
+    pr.cu_seqlens_q = cu_seqlens_q.data_ptr() if cu_seqlens_q is not None else None
+    pr.cu_seqlens_k = cu_seqlens_k.data_ptr() if cu_seqlens_k is not None else None
+    pr.total_q, pr.total_k = total_q, total_k
+    for name, st in (("q_stride", q_stride), ("k_stride", k_stride), ("v_stride", v_stride),
+                     ("o_stride", o_stride)):
+        arr = getattr(pr, name)
+        for i in range(3):
+            arr[i] = int(st[i])
+    pr.dtype = _dtype_code(dtype)
+    pr.causal = int(bool(causal))
+    pr.sm_scale = float(sm_scale or 0.0)
+    pr.smooth_k = int(bool(smooth_k))
+    pr.gscale = GSCALE[gscale]
+    return pr
+
+
+def problem_sizes(pr: _Problem) -> dict:
+    z = _ProblemSizes()
+    _check(lib().sage_fp4_problem_sizes(ctypes.byref(pr), ctypes.byref(z)), "sage_fp4_problem_sizes")
+    return {n: int(getattr(z, n)) for n, _ in _ProblemSizes._fields_}
+
+
+def quantize(pr: _Problem, q, k, v) -> dict:
+    """K statistics, second-level maxima and FP4 quantization of a general problem into
+    freshly allocated buffers (returned as uint8 / float32 / int32 tensors)."""
+    z = problem_sizes(pr)
+    dev = q.device
+    buf = {n: torch.empty(max(z[n], 16), dtype=torch.uint8, device=dev) for n in _QZ_FIELDS}
+    scratch = torch.empty(max(z["scratch"], 16), dtype=torch.uint8, device=dev)
+    qz = _Quantized(*[ctypes.c_void_p(buf[n].data_ptr()) for n in _QZ_FIELDS])
+    _check(lib().sage_fp4_quantize(ctypes.byref(pr), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(qz),
+                                   _ptr(scratch), z["scratch"], _stream(dev)), "sage_fp4_quantize")
+    buf["k_mean"] = buf["k_mean"].view(torch.float32)
+    buf["amax"] = buf["amax"].view(torch.float32)
+    buf["seq"] = buf["seq"].view(torch.int32)
+    buf["problem"] = pr
+    return buf
+
+
+def attn_quantized_problem(qz: dict, out: torch.Tensor) -> torch.Tensor:
+    """Fused attention on the output of :func:`quantize` (same problem), into `out`."""
+    pr = qz["problem"]
+    c = _Quantized(*[ctypes.c_void_p(qz[n].data_ptr()) for n in _QZ_FIELDS])
+    _check(lib().sage_fp4_attn_quantized(ctypes.byref(pr), ctypes.byref(c), _ptr(out), _stream(out.device)),
+           "sage_fp4_attn_quantized")
+    return out
+
+
+def _run(pr: _Problem, q, k, v, out, workspace):
+    ws = problem_sizes(pr)["workspace"]
+    if workspace is None or workspace.numel() < ws:
+        workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=q.device)
+    _check(lib().sage_fp4_attn(ctypes.byref(pr), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(workspace),
+                               workspace.numel(), _stream(q.device)), "sage_fp4_attn")
+    return out
+
+
+def _same_kind(q, k, v):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must have the same dtype")
+    if k.shape != v.shape:
+        raise ValueError("k and v must have the same shape")
+
+
+def sageattn_problem(q, k, v, out, tensor_layout: str = "HND", is_causal: bool = False,
+                     sm_scale: Optional[float] = None, smooth_k: bool = True,
+                     gscale: str = "none") -> _Problem:
+    """The problem descriptor :func:`sageattn` passes to the library."""
+    _same_kind(q, k, v)
+    if tensor_layout == "HND":
+        B, Hq, Nq, D = q.shape
+        _, Hkv, Nk, _ = k.shape
+        dims = (0, 1, 2)
+    elif tensor_layout == "NHD":
+        B, Nq, Hq, D = q.shape
+        _, Nk, Hkv, _ = k.shape
+        dims = (0, 2, 1)
+    else:
+        raise ValueError("tensor_layout must be 'HND' or 'NHD'")
+    if k.shape[0] != B or k.shape[-1] != D:
+        raise ValueError("q and k disagree on batch or head dimension")
+    return make_problem(B=B, Hq=Hq, Hkv=Hkv, D=D, Nq=Nq, Nk=Nk, dtype=q.dtype,
+                        q_stride=_strides3(q, dims), k_stride=_strides3(k, dims),
+                        v_stride=_strides3(v, dims), o_stride=_strides3(out, dims), causal=is_causal,
+                        sm_scale=sm_scale, smooth_k=smooth_k, gscale=gscale)
+
+
+def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tensor_layout: str = "HND",
+             is_causal: bool = False, sm_scale: Optional[float] = None, smooth_k: bool = True,
+             gscale: str = "none", out: Optional[torch.Tensor] = None,
+             workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """FP4 attention on [B, H, N, D] ("HND") or [B, N, H, D] ("NHD") tensors with any
+    strides (channels contiguous). k and v may have fewer heads than q (each shared by
+    Hq / Hkv query heads) and a different length (the causal mask then aligns the last
+    query with the last key). gscale adds a second-level FP32 scale per tensor ("tensor")
+    or per (batch, head) ("head")."""
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, device=q.device)
+    pr = sageattn_problem(q, k, v, out, tensor_layout, is_causal, sm_scale, smooth_k, gscale)
+    return _run(pr, q, k, v, out, workspace)
+
+
+def sageattn_varlen_problem(q, k, v, out, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                            max_seqlen_k: int, is_causal: bool = False,
+                            sm_scale: Optional[float] = None, smooth_k: bool = True,
+                            gscale: str = "none") -> _Problem:
+    """The problem descriptor :func:`sageattn_varlen` passes to the library."""
+    _same_kind(q, k, v)
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("packed tensors are [total, H, D]")
+    for t in (cu_seqlens_q, cu_seqlens_k):
+        if t.dtype != torch.int32 or not t.is_cuda or t.dim() != 1 or not t.is_contiguous():
+            raise ValueError("cu_seqlens must be contiguous int32 CUDA tensors")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both hold B + 1 offsets")
+    total_q, Hq, D = q.shape
+    total_k, Hkv, _ = k.shape
+    dims = (0, 1, 0)
+    return make_problem(B=cu_seqlens_q.numel() - 1, Hq=Hq, Hkv=Hkv, D=D, Nq=int(max_seqlen_q),
+                      Nk=int(max_seqlen_k), dtype=q.dtype, q_stride=_strides3(q, dims),
+                      k_stride=_strides3(k, dims), v_stride=_strides3(v, dims),
+                      o_stride=_strides3(out, dims), causal=is_causal, sm_scale=sm_scale,
+                      smooth_k=smooth_k, gscale=gscale, cu_seqlens_q=cu_seqlens_q,
+                      cu_seqlens_k=cu_seqlens_k, total_q=total_q, total_k=total_k)
+
+
+def sageattn_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.Tensor,
+                    cu_seqlens_k: torch.Tensor, max_seqlen_q: int, max_seqlen_k: int,
+                    is_causal: bool = False, sm_scale: Optional[float] = None,
+                    smooth_k: bool = True, gscale: str = "none",
+                    out: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """FP4 attention on packed sequences: q [total_q, Hq, D], k and v [total_k, Hkv, D];
+    sequence b holds tokens cu_seqlens_q[b] .. cu_seqlens_q[b+1] (int32 CUDA tensors of
+    B+1 offsets; a bad table is reported by device_error(), never by a fault). Each
+    sequence is its own problem: its own K mean, causal mask and ("head") scales."""
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, device=q.device)
+    pr = sageattn_varlen_problem(q, k, v, out, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                                 max_seqlen_k, is_causal, sm_scale, smooth_k, gscale)
+    return _run(pr, q, k, v, out, workspace)

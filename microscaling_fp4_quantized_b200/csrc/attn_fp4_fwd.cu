@@ -6,7 +6,10 @@
 // diag(l)^-1 after the last key tile (reply to Q2), and the two-level P~ quantization
 // (per-row factor s1 = rowmax(P~)/(448*6) per key tile, then 16-element E4M3 scales).
 //
-// One CTA per (128-query tile, batch*head); key tiles of 128. Warp roles:
+// One CTA per (128-query tile, query head, sequence); key tiles of 128. Sequences may be
+// packed with different lengths, query heads may share key/value heads (head h reads
+// key/value head h / (Hq / Hkv)), and the causal mask keeps key j <= i + (len_k - len_q)
+// for query i (the last query sees the last key). Warp roles:
 //   warp 0      TMA producer: Q^ + scales once, then K^/V^T tiles + scales into a
 //               3-stage shared-memory ring (cp.async.bulk.tensor / cp.async.bulk).
 //   warp 1      allocates 512 tensor-memory columns; one thread issues the tcgen05
@@ -179,10 +182,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   float* lsum = reinterpret_cast<float*>(smem + L::off_lsum);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int nqt = p.Np / 128;
+  if (seq_table_bad(p.seq)) return;
+  const int bseq = blockIdx.z, hq = blockIdx.y;
+  const SeqInfo si = seq_info(p.seq, bseq);
+  const int nqt = (si.len_q + 127) >> 7;
+  if (static_cast<int>(blockIdx.x) >= nqt) return;  // uniform: before any barrier or allocation
   const int qt = CAUSAL ? (nqt - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
-  const int bh = blockIdx.y;
-  const int nt = CAUSAL ? (qt + 1) : nqt;  // key tiles to visit
+  const int hk = hq / p.group;
+  const int nkt = (si.len_k + 127) >> 7;
+  const int coff = si.len_k - si.len_q;  // causal: query i sees keys j <= i + coff
+  int nt = nkt;                          // key tiles to visit
+  if (CAUSAL) {
+    const int last = qt * 128 + 127 + coff;
+    nt = last < 0 ? 0 : min(nkt, last / 128 + 1);
+  }
+  // Padded rows (TMA coordinates) of this Q tile and of key tile 0; 128-row tiles of
+  // those rows index the scale-factor tiles and the V^T tiles.
+  const int qrow0 = p.Hq * si.prow_q + hq * nqt * 128 + qt * 128;
+  const int ktile0 = (p.Hkv * si.prow_k + hk * nkt * 128) >> 7;
   Ctl ctl{misc + 1, p.err, p.timeout_ns};
 
   if (threadIdx.x == 0) {
@@ -225,8 +242,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (lane == 0 && !(p.debug_flags & kDebugNoLoads)) {
       const uint32_t sq = sbase + L::off_q;
       mbar_arrive_expect_tx(bar(B_QFULL), L::kQBytes + L::kSfQKBytes);
-      tma_load_2d(sq, &tm_q, 0, bh * p.Np + qt * 128, bar(B_QFULL));
-      bulk_load(sbase + L::off_sfq, p.q_sf + (static_cast<size_t>(bh) * nqt + qt) * L::kSfQKBytes,
+      tma_load_2d(sq, &tm_q, 0, qrow0, bar(B_QFULL));
+      bulk_load(sbase + L::off_sfq, p.q_sf + static_cast<size_t>(qrow0 >> 7) * L::kSfQKBytes,
                 L::kSfQKBytes, bar(B_QFULL));
       int issued = 0;
       for (int j = 0; j < nt; ++j) {
@@ -234,12 +251,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!wait_bar(bar(B_KVEMPTY + st), ((j / kStages) & 1) ^ 1, ctl)) break;
         const uint32_t sst = sbase + L::off_stage + st * L::kStageBytes;
         mbar_arrive_expect_tx(bar(B_KFULL + st), L::kKBytes + L::kSfQKBytes);
-        tma_load_2d(sst + L::st_k, &tm_k, 0, bh * p.Np + j * 128, bar(B_KFULL + st));
-        bulk_load(sst + L::st_sfk, p.k_sf + (static_cast<size_t>(bh) * nqt + j) * L::kSfQKBytes,
+        tma_load_2d(sst + L::st_k, &tm_k, 0, (ktile0 + j) * 128, bar(B_KFULL + st));
+        bulk_load(sst + L::st_sfk, p.k_sf + static_cast<size_t>(ktile0 + j) * L::kSfQKBytes,
                   L::kSfQKBytes, bar(B_KFULL + st));
         mbar_arrive_expect_tx(bar(B_VFULL + st), L::kVBytes + L::kSfVBytes);
-        tma_load_2d(sst + L::st_v, &tm_v, j * 64, bh * D, bar(B_VFULL + st));
-        bulk_load(sst + L::st_sfv, p.vt_sf + (static_cast<size_t>(bh) * nqt + j) * L::kSfVBytes,
+        tma_load_2d(sst + L::st_v, &tm_v, 0, (ktile0 + j) * D, bar(B_VFULL + st));
+        bulk_load(sst + L::st_sfv, p.vt_sf + static_cast<size_t>(ktile0 + j) * L::kSfVBytes,
                   L::kSfVBytes, bar(B_VFULL + st));
         issued = j + 1;
       }
@@ -316,7 +333,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int r = quad * 32 + lane;
     const int qrow = qt * 128 + r;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const float xs = p.sm_scale_log2;
+    float xs = p.sm_scale_log2, gv = 1.0f;
+    if (p.amax != nullptr) {
+      // Second-level scales fold into the score scale (Q and K) and the output (V).
+      const bool head = p.gscale == kGscaleHead;
+      const float gq = second_level_scale(p.amax[head ? bseq * p.Hq + hq : 0]);
+      const float gk = second_level_scale(p.amax[p.amax_stride + (head ? bseq * p.Hkv + hk : 0)]);
+      gv = second_level_scale(p.amax[2 * p.amax_stride + (head ? bseq * p.Hkv + hk : 0)]);
+      xs = xs * gq * gk;
+    }
     float o[DH];
 #pragma unroll
     for (int d = 0; d < DH; ++d) o[d] = 0.0f;
@@ -368,12 +393,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(sr[c][i]);
       const int kbase = j * 128 + 64 * h;
-      const bool need_mask = CAUSAL ? (j == nt - 1) : (j * 128 + 128 > p.N);
+      const bool need_mask = (j * 128 + 128 > si.len_k) || (CAUSAL && j * 128 + 127 > qt * 128 + coff);
       if (need_mask) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const int key = kbase + c;
-          if (key >= p.N || (CAUSAL && key > qrow)) s[c] = -INFINITY;
+          if (key >= si.len_k || (CAUSAL && key > qrow + coff)) s[c] = -INFINITY;
         }
       }
       // Block maxima of the raw scores (sm_scale > 0, so they order like P~).
@@ -392,6 +417,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (lane == 0) mbar_arrive(bar(B_XCH + (j & 1)));
       if (!__all_sync(0xffffffffu, wait_bar(bar(B_XCH + (j & 1)), (j >> 1) & 1, ctl))) { ok = false; break; }
       const float tm = fmaxf(hm, xb[(1 - h) * 128 + r]);
+      // A row can see no key of this tile (causal with len_q > len_k, or a mask offset
+      // that is not a multiple of 128): it then adds nothing, and its P^ codes are 0.
+      const bool empty = tm == -INFINITY;
 
       const float tmx = tm * xs;
       // Reference max: it moves only when the tile max exceeds it by more than 8 (log2
@@ -401,8 +429,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const bool move = tmx > m_run + 8.0f;  // always true on the first tile (m_run = -inf)
       const float m_new = move ? tmx : m_run;
       const float alpha = move ? ex2_approx(m_run - m_new) : 1.0f;
-      const float rfac = ex2_approx(tmx - m_new);  // rowmax of P~ in this tile (<= 2^8)
+      const float rfac = empty ? 0.0f : ex2_approx(tmx - m_new);  // rowmax of P~ in this tile (<= 2^8)
       const float s1 = rfac * (1.0f / 2688.0f);
+      const float tref = empty ? 0.0f : tmx;
 
       // Per-16 scales of P2 = P~ / s1 = exp2(S*xs - tmx) * 2688. The division by the
       // decoded block scale is folded into the exp2 argument: v = exp2(S*xs - nb) = P2 / s.
@@ -412,14 +441,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       uint32_t sfw = 0, zero_blocks = 0;
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
-        const float amax = ex2_approx(fmaf(bm[b], xs, -tmx)) * 2688.0f;
+        const float amax = ex2_approx(fmaf(bm[b], xs, -tref)) * 2688.0f;
         const uint32_t sbyte = f32_to_e4m3(amax * (1.0f / 6.0f));
         const float sdec = e4m3_to_f32(sbyte);
         if (sdec > 0.0f) {
-          nb[b] = -(tmx + lg2_approx(sdec) - 11.392317422778761f);  // log2(2688)
+          nb[b] = -(tref + lg2_approx(sdec) - 11.392317422778761f);  // log2(2688)
           mult[b] = sdec * (1.0f / 2688.0f);
         } else {
-          nb[b] = -tmx;
+          nb[b] = -tref;
           mult[b] = 1.0f;
           zero_blocks |= 1u << b;
         }
@@ -470,16 +499,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       alpha_prev = alpha;
       s1_prev = s1;
     }
-    if (ok) ok = correct(nt - 1, alpha_prev, s1_prev);
+    if (ok && nt > 0) ok = correct(nt - 1, alpha_prev, s1_prev);
     if (ok) {
       lsum[h * 128 + r] = l_half;
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_LSUM));
       ok = __all_sync(0xffffffffu, wait_bar(bar(B_LSUM), 0, ctl));
     }
-    if (ok && qrow < p.N) {
-      const float il = 1.0f / (l_half + lsum[(1 - h) * 128 + r]);
-      const size_t base = (static_cast<size_t>(bh) * p.N + qrow) * D + DH * h;
+    if (ok && qrow < si.len_q) {
+      // A row that saw no key (l = 0) is written as 0.
+      const float l = l_half + lsum[(1 - h) * 128 + r];
+      const float il = l > 0.0f ? gv / l : 0.0f;
+      const size_t base = static_cast<size_t>(static_cast<int64_t>(bseq) * p.so.b + static_cast<int64_t>(hq) * p.so.h +
+                                              (static_cast<int64_t>(si.tok_q) + qrow) * p.so.n) + DH * h;
 #pragma unroll
       for (int d = 0; d < DH; d += 8) {
         float v8[8];
@@ -592,19 +624,20 @@ static int attn_smem_bytes() {
 }
 
 template <int D, bool CAUSAL>
-static cudaError_t launch_attn_t(const TensorMaps& m, const AttnParams& p, cudaStream_t stream) {
+static cudaError_t launch_attn_t(const TensorMaps& m, const AttnParams& p, int tiles_q, cudaStream_t stream) {
   const int smem = attn_smem_bytes<D>();
   cudaError_t e = cudaFuncSetAttribute(attn_fp4_fwd_kernel<D, CAUSAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.Np / 128, p.BH);
+  dim3 grid(tiles_q, p.Hq, p.B);
   attn_fp4_fwd_kernel<D, CAUSAL><<<grid, kAttnThreads, smem, stream>>>(m.q, m.k, m.v, p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_attention(const TensorMaps& m, const AttnParams& p, cudaStream_t stream) {
-  if (p.BH == 0 || p.N == 0) return cudaSuccess;
-  if (p.D == 64) return p.causal ? launch_attn_t<64, true>(m, p, stream) : launch_attn_t<64, false>(m, p, stream);
-  return p.causal ? launch_attn_t<128, true>(m, p, stream) : launch_attn_t<128, false>(m, p, stream);
+cudaError_t launch_attention(const TensorMaps& m, const AttnParams& p, int tiles_q, cudaStream_t stream) {
+  if (p.B == 0 || p.Hq == 0 || tiles_q == 0) return cudaSuccess;
+  if (p.D == 64)
+    return p.causal ? launch_attn_t<64, true>(m, p, tiles_q, stream) : launch_attn_t<64, false>(m, p, tiles_q, stream);
+  return p.causal ? launch_attn_t<128, true>(m, p, tiles_q, stream) : launch_attn_t<128, false>(m, p, tiles_q, stream);
 }
 
 template <int D>
@@ -618,7 +651,7 @@ static cudaError_t launch_scores_t(const TensorMaps& m, const AttnParams& p, cud
 }
 
 cudaError_t launch_qk_scores(const TensorMaps& m, const AttnParams& p, cudaStream_t stream) {
-  if (p.BH == 0 || p.N == 0) return cudaSuccess;
+  if (p.BH == 0 || p.Np == 0) return cudaSuccess;
   return p.D == 64 ? launch_scores_t<64>(m, p, stream) : launch_scores_t<128>(m, p, stream);
 }
 

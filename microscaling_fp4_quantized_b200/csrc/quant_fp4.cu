@@ -1,16 +1,24 @@
 // Quantization kernels of the FP4 attention forward (sm_100a):
-//   kmean_partial_kernel : binary64 column sums of K over 512-token chunks
-//   quant_kernel         : Q, K - mean and V^T -> packed E2M1 codes + UE4M3 scale tiles
+//   seq_plan_kernel  : packed sequences only -- checks the sequence table and prefix-sums
+//                      the padded (multiple-of-128) lengths
+//   stats_kernel     : per 512-token chunk: binary64 column sums of K; with a second-level
+//                      scale also the column maxima / minima of K and the maxima of |Q|, |V|
+//   finalize_kernel  : per (sequence, head): the K mean and the second-level maxima
+//   quant_kernel     : Q, K - mean and V^T -> packed E2M1 codes + UE4M3 scale tiles
 //
 // The block rule follows the microscaling FP4 statement of SageAttention3 (arXiv
 // 2505.11594, abstract): per 16 consecutive elements, s = E4M3(absmax / 6) and
 // code = E2M1(x / s), both round-to-nearest-even with saturation; "smoothing K"
 // (SageAttention OpenReview thread, reply to W1) subtracts the per-channel token mean
-// of K first. Every arithmetic step is IEEE binary32 with RNE (true divisions, no
+// of K first. The optional second-level scale (NVFP4's FP32 factor, named on the
+// author page, "TetraJet-v2" abstract) divides a whole tensor, or one head of one
+// sequence, by g = amax / 2688 before the block rule -- the same two-level shape the
+// method gives P~. Every arithmetic step is IEEE binary32 with RNE (true divisions, no
 // reciprocal), so codes and scale bytes are reproducible bit for bit.
 //
-// Both kernels are HBM-bound: 16-byte coalesced loads, tiles of 128 tokens, scale
-// factors and V^T codes staged in shared memory and written out as 16-byte chunks.
+// All four kernels are HBM-bound (or tiny): 16-byte coalesced loads, tiles of 128
+// tokens, scale factors and V^T codes staged in shared memory and written out as
+// 16-byte chunks; V^T is stored tile-major (one contiguous D x 64-byte block per tile).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -59,42 +67,232 @@ __device__ __forceinline__ uint32_t encode8(const float (&x)[8], float s) {
   return w;
 }
 
+// Address of element (b, h, token) of a [.., D] input whose channels are contiguous.
+__device__ __forceinline__ const char* row_ptr(const void* base, const Strides& s, int b, int h, int64_t tok) {
+  return static_cast<const char*>(base) + (static_cast<int64_t>(b) * s.b + static_cast<int64_t>(h) * s.h + tok * s.n) * 2;
+}
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x / 32, nw = blockDim.x / 32;
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  float r = 0.0f;
+  for (int i = 0; i < nw; ++i) r = fmaxf(r, red[i]);
+  return r;
+}
+
+__device__ __forceinline__ void amax_store(float* slot, int mode, float a) {
+  if (mode == kGscaleTensor) atomicMax(reinterpret_cast<unsigned int*>(slot), __float_as_uint(a));
+  else *slot = a;
+}
+
 constexpr int kThreads = 256;
-constexpr int kMeanChunk = 512;  // tokens per K-mean partial
+constexpr int kChunk = 512;  // tokens per statistics chunk
 
 }  // namespace
 
-// grid (nsplit, BH); partial[bh, split, d] = sum over tokens of the chunk, binary64.
+// One CTA. Checks cu_q / cu_k (start at 0, non-decreasing, end at the packed totals,
+// no sequence longer than its stated maximum) and writes the exclusive prefix sums of
+// the padded lengths; a failed check sets *bad and the device error bit instead.
+__global__ void __launch_bounds__(1024) seq_plan_kernel(QuantParams p) {
+  __shared__ long long wq[32], wk[32];
+  __shared__ int s_bad;
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  if (t == 0) s_bad = 0;
+  __syncthreads();
+  const int B = p.B;
+  const int per = (B + 1023) / 1024;
+  const int b0 = min(B, t * per), b1 = min(B, b0 + per);
+  long long sq = 0, sk = 0;
+  int bad = 0;
+  for (int b = b0; b < b1; ++b) {
+    const int lq = p.seq.cu_q[b + 1] - p.seq.cu_q[b];
+    const int lk = p.seq.cu_k[b + 1] - p.seq.cu_k[b];
+    if (lq < 0 || lk < 0 || lq > p.seq.Nq || lk > p.seq.Nk) bad = 1;
+    sq += (max(lq, 0) + 127) / 128 * 128;
+    sk += (max(lk, 0) + 127) / 128 * 128;
+  }
+  if (t == 0 && (p.seq.cu_q[0] != 0 || p.seq.cu_k[0] != 0 || p.seq.cu_q[B] != p.total_q ||
+                 p.seq.cu_k[B] != p.total_k))
+    bad = 1;
+  if (bad) atomicOr(&s_bad, 1);
+  // Block-wide inclusive scan of (sq, sk).
+  long long iq = sq, ik = sk;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long a = __shfl_up_sync(0xffffffffu, iq, o), c = __shfl_up_sync(0xffffffffu, ik, o);
+    if (lane >= o) {
+      iq += a;
+      ik += c;
+    }
+  }
+  if (lane == 31) {
+    wq[w] = iq;
+    wk[w] = ik;
+  }
+  __syncthreads();
+  long long oq = 0, ok = 0;
+  for (int i = 0; i < w; ++i) {
+    oq += wq[i];
+    ok += wk[i];
+  }
+  long long eq = oq + iq - sq, ek = ok + ik - sk;  // exclusive prefix of this thread's range
+  __syncthreads();
+  if (s_bad) {
+    if (t == 0) {
+      *p.bad_out = 1u;
+      atomicOr(p.err, kDevErrSeqlens);
+    }
+    return;
+  }
+  for (int b = b0; b < b1; ++b) {
+    p.pad_q_out[b] = static_cast<int32_t>(eq);
+    p.pad_k_out[b] = static_cast<int32_t>(ek);
+    eq += (p.seq.cu_q[b + 1] - p.seq.cu_q[b] + 127) / 128 * 128;
+    ek += (p.seq.cu_k[b + 1] - p.seq.cu_k[b] + 127) / 128 * 128;
+  }
+  if (b1 == B) {
+    p.pad_q_out[B] = static_cast<int32_t>(eq);
+    p.pad_k_out[B] = static_cast<int32_t>(ek);
+  }
+  if (t == 0) *p.bad_out = 0u;
+}
+
+// grid (nsplit, Hq, B): chunk `split` of sequence b, head h.
+//   K (h < Hkv): ksum[bh, split, d] = sum over the chunk's tokens, binary64; with a
+//     second-level scale also kmax / kmin per channel.
+//   Q (h < Hq) and V (h < Hkv), second-level scale only: max |x| over the chunk.
 template <int D>
-__global__ void __launch_bounds__(kThreads) kmean_partial_kernel(QuantParams p) {
+__global__ void __launch_bounds__(kThreads) stats_kernel(QuantParams p) {
   constexpr int CPR = D / 8;          // 16-byte chunks per row
   constexpr int RG = kThreads / CPR;  // row groups
   __shared__ double red[RG][D];
+  __shared__ float redmx[RG][D], redmn[RG][D];
+  __shared__ float redw[kThreads / 32];
+  if (seq_table_bad(p.seq)) return;
   const int t = threadIdx.x, c = t % CPR, rg = t / CPR;
-  const int bh = blockIdx.y;
-  const int n0 = blockIdx.x * kMeanChunk;
-  const int n1 = min(n0 + kMeanChunk, p.N);
-  const char* base = static_cast<const char*>(p.k) + (static_cast<size_t>(bh) * p.N) * D * 2;
-  double acc[8];
+  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const SeqInfo si = seq_info(p.seq, b);
+  const bool gs = p.gscale != kGscaleNone;
+  if (gs && p.gscale == kGscaleTensor && split == 0 && h == 0 && b == 0 && t < 3) p.amax[t * p.amax_stride] = 0.0f;
+  const int n0 = split * kChunk;
+
+  if (h < p.Hkv && (p.smooth_k || gs) && n0 < si.len_k) {
+    const int n1 = min(n0 + kChunk, si.len_k);
+    double acc[8];
+    float mx[8], mn[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.0;
-  for (int n = n0 + rg; n < n1; n += RG) {
-    float x[8];
-    unpack8(ld_nc_16(base + (static_cast<size_t>(n) * D + c * 8) * 2), p.dtype, x);
+    for (int e = 0; e < 8; ++e) {
+      acc[e] = 0.0;
+      mx[e] = -INFINITY;
+      mn[e] = INFINITY;
+    }
+    for (int n = n0 + rg; n < n1; n += RG) {
+      float x[8];
+      unpack8(ld_nc_16(row_ptr(p.k, p.sk, b, h, static_cast<int64_t>(si.tok_k) + n) + c * 16), p.dtype, x);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += static_cast<double>(x[e]);
+      for (int e = 0; e < 8; ++e) {
+        acc[e] += static_cast<double>(x[e]);
+        mx[e] = fmaxf(mx[e], x[e]);
+        mn[e] = fminf(mn[e], x[e]);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      red[rg][c * 8 + e] = acc[e];
+      redmx[rg][c * 8 + e] = mx[e];
+      redmn[rg][c * 8 + e] = mn[e];
+    }
+    __syncthreads();
+    const size_t base = (static_cast<size_t>(b * p.Hkv + h) * p.nsplit + split) * D;
+    for (int d = t; d < D; d += kThreads) {
+      double s = 0.0;
+      float a = -INFINITY, z = INFINITY;
+      for (int g = 0; g < RG; ++g) {
+        s += red[g][d];
+        a = fmaxf(a, redmx[g][d]);
+        z = fminf(z, redmn[g][d]);
+      }
+      p.ksum[base + d] = s;
+      if (gs) {
+        p.kmax[base + d] = a;
+        p.kmin[base + d] = z;
+      }
+    }
   }
+  if (!gs) return;
+  for (int job = 0; job < 2; ++job) {  // 0: Q, 1: V
+    const int H = job == 0 ? p.Hq : p.Hkv;
+    const int len = job == 0 ? si.len_q : si.len_k;
+    if (h >= H || n0 >= len) continue;
+    const int n1 = min(n0 + kChunk, len);
+    const void* src = job == 0 ? p.q : p.v;
+    const Strides& st = job == 0 ? p.sq : p.sv;
+    const int tok = job == 0 ? si.tok_q : si.tok_k;
+    float a = 0.0f;
+    for (int n = n0 + rg; n < n1; n += RG) {
+      float x[8];
+      unpack8(ld_nc_16(row_ptr(src, st, b, h, static_cast<int64_t>(tok) + n) + c * 16), p.dtype, x);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) red[rg][c * 8 + e] = acc[e];
-  __syncthreads();
-  for (int d = t; d < D; d += kThreads) {
-    double s = 0.0;
-    for (int g = 0; g < RG; ++g) s += red[g][d];
-    p.partial[(static_cast<size_t>(bh) * p.nsplit + blockIdx.x) * D + d] = s;
+      for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(x[e]));
+    }
+    a = block_max(a, redw);
+    if (t == 0) (job == 0 ? p.qamax : p.vamax)[static_cast<size_t>(b * H + h) * p.nsplit + split] = a;
   }
 }
 
-// grid (Np/128, BH, 3): z = 0 quantizes Q rows, 1 quantizes K rows (smoothed), 2 V^T.
+// grid (Hq, B), D threads: the K mean of (sequence b, key/value head h) and the
+// second-level maxima of Q (head h) and of K - mean and V (head h).
+template <int D>
+__global__ void __launch_bounds__(D) finalize_kernel(QuantParams p) {
+  __shared__ float redw[D / 32];
+  if (seq_table_bad(p.seq)) return;
+  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  const SeqInfo si = seq_info(p.seq, b);
+  const bool gs = p.gscale != kGscaleNone;
+  if (h < p.Hkv) {
+    const int ns = (si.len_k + kChunk - 1) / kChunk;
+    const size_t base = static_cast<size_t>(b * p.Hkv + h) * p.nsplit * D + d;
+    float mu = 0.0f;
+    if (p.smooth_k && si.len_k > 0) {
+      double s = 0.0;
+      for (int g = 0; g < ns; ++g) s += p.ksum[base + static_cast<size_t>(g) * D];
+      mu = static_cast<float>(s / static_cast<double>(si.len_k));
+    }
+    p.k_mean[static_cast<size_t>(b * p.Hkv + h) * D + d] = mu;
+    if (gs) {
+      float mx = -INFINITY, mn = INFINITY, av = 0.0f;
+      for (int g = 0; g < ns; ++g) {
+        mx = fmaxf(mx, p.kmax[base + static_cast<size_t>(g) * D]);
+        mn = fminf(mn, p.kmin[base + static_cast<size_t>(g) * D]);
+      }
+      // Rounding is monotone, so max |fp32(k - mu)| over the tokens is reached at the
+      // channel's largest or smallest k.
+      float ak = si.len_k > 0 ? fmaxf(fabsf(__fsub_rn(mx, mu)), fabsf(__fsub_rn(mn, mu))) : 0.0f;
+      ak = block_max(ak, redw);
+      for (int g = d; g < ns; g += D) av = fmaxf(av, p.vamax[static_cast<size_t>(b * p.Hkv + h) * p.nsplit + g]);
+      av = block_max(av, redw);
+      if (d == 0) {
+        const int i = p.gscale == kGscaleHead ? b * p.Hkv + h : 0;
+        amax_store(p.amax + p.amax_stride + i, p.gscale, ak);
+        amax_store(p.amax + 2 * p.amax_stride + i, p.gscale, av);
+      }
+    }
+  }
+  if (gs && h < p.Hq) {
+    const int ns = (si.len_q + kChunk - 1) / kChunk;
+    float aq = 0.0f;
+    for (int g = d; g < ns; g += D) aq = fmaxf(aq, p.qamax[static_cast<size_t>(b * p.Hq + h) * p.nsplit + g]);
+    aq = block_max(aq, redw);
+    if (d == 0) amax_store(p.amax + (p.gscale == kGscaleHead ? b * p.Hq + h : 0), p.gscale, aq);
+  }
+}
+
+// grid (3 * tiles, Hq, B): x = 3 * tile + job; job 0 quantizes Q rows, 1 K rows
+// (smoothed), 2 V^T. CTAs past a sequence's tiles or heads return at once.
 template <int D>
 __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
   constexpr int CPR = D / 8;
@@ -102,41 +300,48 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
   constexpr int kCodeRow = 80;             // padded V^T code staging row (64 used)
   constexpr int kSfBytesQK = (D / 64) * 512;
   __shared__ __align__(16) uint8_t smem[128 * kVRowBytes + D * kCodeRow + 1024 + D * 4];
+  if (seq_table_bad(p.seq)) return;
   const int t = threadIdx.x;
-  const int bh = blockIdx.y;
-  const int tile = blockIdx.x;
-  const int row0 = tile * 128;
-  const int job = blockIdx.z;
-  const int ntiles = p.Np / 128;
+  const int job = blockIdx.x % 3, tile = blockIdx.x / 3, h = blockIdx.y, b = blockIdx.z;
+  const int H = job == 0 ? p.Hq : p.Hkv;
+  if (h >= H) return;
+  const SeqInfo si = seq_info(p.seq, b);
+  const int len = job == 0 ? si.len_q : si.len_k;
+  const int ntile = (len + 127) >> 7;
+  if (tile >= ntile) return;
+  const int prow = job == 0 ? si.prow_q : si.prow_k;
+  const int64_t tok0 = static_cast<int64_t>(job == 0 ? si.tok_q : si.tok_k) + tile * 128;
+  const int64_t row0 = static_cast<int64_t>(H) * prow + static_cast<int64_t>(h) * ntile * 128 + tile * 128;
+  const int64_t T = row0 >> 7;  // scale-factor / V^T tile index
+  const int rows = min(128, len - tile * 128);
+  const bool gs = p.gscale != kGscaleNone;
+  float g = 1.0f;
+  if (gs) g = second_level_scale(p.amax[job * p.amax_stride + (p.gscale == kGscaleHead ? b * H + h : 0)]);
 
   if (job < 2) {
     uint8_t* sfbuf = smem;                                  // kSfBytesQK
     float* mu = reinterpret_cast<float*>(smem + 1024);      // D floats
     const bool smooth = (job == 1) && p.smooth_k;
-    for (int d = t; d < D; d += kThreads) {
-      float m = 0.0f;
-      if (smooth) {
-        double s = 0.0;
-        for (int g = 0; g < p.nsplit; ++g) s += p.partial[(static_cast<size_t>(bh) * p.nsplit + g) * D + d];
-        m = static_cast<float>(s / static_cast<double>(p.N));
-        if (tile == 0 && p.k_mean != nullptr) p.k_mean[static_cast<size_t>(bh) * D + d] = m;
-      }
-      mu[d] = m;
-    }
+    for (int d = t; d < D; d += kThreads)
+      mu[d] = smooth ? p.k_mean[static_cast<size_t>(b * p.Hkv + h) * D + d] : 0.0f;
     for (int i = t; i < kSfBytesQK / 16; i += kThreads) reinterpret_cast<uint4*>(sfbuf)[i] = make_uint4(0, 0, 0, 0);
     __syncthreads();
-    const char* src = static_cast<const char*>(job == 0 ? p.q : p.k) + static_cast<size_t>(bh) * p.N * D * 2;
-    uint8_t* dst = (job == 0 ? p.q_fp4 : p.k_fp4) + static_cast<size_t>(bh) * p.Np * (D / 2);
+    const void* src = job == 0 ? p.q : p.k;
+    const Strides& st = job == 0 ? p.sq : p.sk;
+    uint8_t* dst = (job == 0 ? p.q_fp4 : p.k_fp4) + row0 * (D / 2);
 #pragma unroll 2
-    for (int g = t; g < 128 * CPR; g += kThreads) {
-      const int rl = g / CPR, c = g % CPR;
-      const int n = row0 + rl;
+    for (int gi = t; gi < 128 * CPR; gi += kThreads) {
+      const int rl = gi / CPR, c = gi % CPR;
       float x[8];
-      if (n < p.N) {
-        unpack8(ld_nc_16(src + (static_cast<size_t>(n) * D + c * 8) * 2), p.dtype, x);
+      if (rl < rows) {
+        unpack8(ld_nc_16(row_ptr(src, st, b, h, tok0 + rl) + c * 16), p.dtype, x);
         if (smooth) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], mu[c * 8 + e]);
+        }
+        if (gs) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = __fdiv_rn(x[e], g);
         }
       } else {
 #pragma unroll
@@ -149,14 +354,14 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
       const uint32_t sb = f32_to_e4m3(__fdiv_rn(a, 6.0f));
       const float s = e4m3_to_f32(sb);
       const uint32_t w = encode8(x, s);
-      *reinterpret_cast<uint32_t*>(dst + static_cast<size_t>(n) * (D / 2) + c * 4) = w;
+      *reinterpret_cast<uint32_t*>(dst + static_cast<size_t>(rl) * (D / 2) + c * 4) = w;
       if ((c & 1) == 0) {
         const int col = c * 8;
         sfbuf[(col / 64) * 512 + (rl % 32) * 16 + (rl / 32) * 4 + (col % 64) / 16] = static_cast<uint8_t>(sb);
       }
     }
     __syncthreads();
-    uint8_t* sf_out = (job == 0 ? p.q_sf : p.k_sf) + (static_cast<size_t>(bh) * ntiles + tile) * kSfBytesQK;
+    uint8_t* sf_out = (job == 0 ? p.q_sf : p.k_sf) + T * kSfBytesQK;
     for (int i = t; i < kSfBytesQK / 16; i += kThreads)
       reinterpret_cast<uint4*>(sf_out)[i] = reinterpret_cast<const uint4*>(sfbuf)[i];
     return;
@@ -166,13 +371,11 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
   uint8_t* vtile = smem;                                // 128 x kVRowBytes
   uint8_t* cbuf = smem + 128 * kVRowBytes;              // D x kCodeRow
   uint8_t* sfbuf = cbuf + D * kCodeRow;                 // 1024
-  const char* src = static_cast<const char*>(p.v) + static_cast<size_t>(bh) * p.N * D * 2;
   for (int i = t; i < 1024 / 16; i += kThreads) reinterpret_cast<uint4*>(sfbuf)[i] = make_uint4(0, 0, 0, 0);
-  for (int g = t; g < 128 * CPR; g += kThreads) {
-    const int rl = g / CPR, c = g % CPR;
-    const int n = row0 + rl;
+  for (int gi = t; gi < 128 * CPR; gi += kThreads) {
+    const int rl = gi / CPR, c = gi % CPR;
     uint4 raw = make_uint4(0, 0, 0, 0);
-    if (n < p.N) raw = ld_nc_16(src + (static_cast<size_t>(n) * D + c * 8) * 2);
+    if (rl < rows) raw = ld_nc_16(row_ptr(p.v, p.sv, b, h, tok0 + rl) + c * 16);
     *reinterpret_cast<uint4*>(vtile + rl * kVRowBytes + c * 16) = raw;
   }
   __syncthreads();
@@ -181,9 +384,10 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
     float x[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const uint16_t h = *reinterpret_cast<const uint16_t*>(vtile + (tb * 16 + i) * kVRowBytes + d * 2);
-      x[i] = (p.dtype == kDtypeBF16) ? __uint_as_float(static_cast<uint32_t>(h) << 16)
-                                     : __half2float(__ushort_as_half(h));
+      const uint16_t hv = *reinterpret_cast<const uint16_t*>(vtile + (tb * 16 + i) * kVRowBytes + d * 2);
+      x[i] = (p.dtype == kDtypeBF16) ? __uint_as_float(static_cast<uint32_t>(hv) << 16)
+                                     : __half2float(__ushort_as_half(hv));
+      if (gs) x[i] = __fdiv_rn(x[i], g);
     }
     float a = 0.0f;
 #pragma unroll
@@ -201,30 +405,44 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
     sfbuf[(tb / 4) * 512 + (d % 32) * 16 + (d / 32) * 4 + (tb % 4)] = static_cast<uint8_t>(sb);
   }
   __syncthreads();
-  uint8_t* vt = p.vt_fp4 + static_cast<size_t>(bh) * D * (p.Np / 2) + tile * 64;
-  for (int g = t; g < D * 4; g += kThreads) {
-    const int d = g / 4, k = g % 4;
-    *reinterpret_cast<uint4*>(vt + static_cast<size_t>(d) * (p.Np / 2) + k * 16) =
-        *reinterpret_cast<const uint4*>(cbuf + d * kCodeRow + k * 16);
+  uint8_t* vt = p.vt_fp4 + T * (D * 64);
+  for (int gi = t; gi < D * 4; gi += kThreads) {
+    const int d = gi / 4, k = gi % 4;
+    *reinterpret_cast<uint4*>(vt + d * 64 + k * 16) = *reinterpret_cast<const uint4*>(cbuf + d * kCodeRow + k * 16);
   }
-  uint8_t* sf_out = p.vt_sf + (static_cast<size_t>(bh) * ntiles + tile) * 1024;
+  uint8_t* sf_out = p.vt_sf + T * 1024;
   for (int i = t; i < 1024 / 16; i += kThreads)
     reinterpret_cast<uint4*>(sf_out)[i] = reinterpret_cast<const uint4*>(sfbuf)[i];
 }
 
-cudaError_t launch_quantize(const QuantParams& p, cudaStream_t stream) {
-  if (p.BH == 0 || p.N == 0) return cudaSuccess;
-  const int ntiles = p.Np / 128;
-  if (p.smooth_k) {
-    dim3 g1(p.nsplit, p.BH);
-    if (p.D == 64) kmean_partial_kernel<64><<<g1, kThreads, 0, stream>>>(p);
-    else kmean_partial_kernel<128><<<g1, kThreads, 0, stream>>>(p);
+cudaError_t launch_quantize(const QuantParams& p, const QuantLaunch& l, cudaStream_t stream) {
+  if (p.B == 0 || p.Hq == 0) return cudaSuccess;
+  if (p.seq.cu_q != nullptr) {
+    seq_plan_kernel<<<1, 1024, 0, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  dim3 g2(ntiles, p.BH, 3);
-  if (p.D == 64) quant_kernel<64><<<g2, kThreads, 0, stream>>>(p);
-  else quant_kernel<128><<<g2, kThreads, 0, stream>>>(p);
+  const bool gs = p.gscale != kGscaleNone;
+  if ((p.smooth_k || gs) && p.nsplit > 0) {
+    dim3 g1(p.nsplit, p.Hq, p.B);
+    if (p.D == 64) stats_kernel<64><<<g1, kThreads, 0, stream>>>(p);
+    else stats_kernel<128><<<g1, kThreads, 0, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  // The finalize pass writes the K mean (zeros without smoothing) and the maxima.
+  if (p.k_mean != nullptr || gs) {
+    dim3 g2(p.Hq, p.B);
+    if (p.D == 64) finalize_kernel<64><<<g2, 64, 0, stream>>>(p);
+    else finalize_kernel<128><<<g2, 128, 0, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const int tiles = l.tiles_q > l.tiles_k ? l.tiles_q : l.tiles_k;
+  if (tiles == 0) return cudaSuccess;
+  dim3 g3(3 * tiles, p.Hq, p.B);
+  if (p.D == 64) quant_kernel<64><<<g3, kThreads, 0, stream>>>(p);
+  else quant_kernel<128><<<g3, kThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -84,146 +85,260 @@ sage_status_t make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool valid_dtype(int d) { return d == SAGE_BF16 || d == SAGE_F16; }
+int64_t round128(int64_t x) { return (x + 127) / 128 * 128; }
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
-struct Shape {
-  int64_t BH, N, Np, D, nsplit;
-  bool empty;
+// A checked problem with everything derived from it.
+struct Prob {
+  sage_fp4_problem_t u;  // the caller's description (sm_scale resolved)
+  bool packed, empty, gs;
+  int64_t rows_q, rows_k;  // padded token rows per head (packed: an upper bound)
+  int tiles_q, tiles_k, nsplit;
 };
 
-sage_status_t check_shape(int B, int H, int N, int D, Shape* s) {
-  if (B < 0 || H < 0 || N < 0) return SAGE_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
-  s->BH = static_cast<int64_t>(B) * H;
-  s->N = N;
-  s->Np = (static_cast<int64_t>(N) + 127) / 128 * 128;
-  s->D = D;
-  s->nsplit = (static_cast<int64_t>(N) + 511) / 512;
-  s->empty = (s->BH == 0 || N == 0);
-  if (s->empty) return SAGE_OK;
-  // Grid y/z limits and 32-bit TMA coordinates / element counts.
-  if (s->BH > 65535 || s->BH * s->Np >= (int64_t(1) << 31) || s->BH * s->Np * D >= (int64_t(1) << 33))
+sage_status_t check_problem(const sage_fp4_problem_t* in, Prob* p) {
+  if (in == nullptr) return SAGE_ERR_INVALID_ARG;
+  const sage_fp4_problem_t& u = *in;
+  p->u = u;
+  if (u.B < 0 || u.Hq < 0 || u.Hkv < 0 || u.Nq < 0 || u.Nk < 0) return SAGE_ERR_INVALID_ARG;
+  if (u.D != 64 && u.D != 128) return SAGE_ERR_UNSUPPORTED;
+  if (!valid_dtype(u.dtype)) return SAGE_ERR_INVALID_ARG;
+  if (u.gscale != SAGE_GSCALE_NONE && u.gscale != SAGE_GSCALE_TENSOR && u.gscale != SAGE_GSCALE_HEAD)
+    return SAGE_ERR_INVALID_ARG;
+  if (!std::isfinite(u.sm_scale)) return SAGE_ERR_INVALID_ARG;
+  p->u.sm_scale = u.sm_scale > 0.0f ? u.sm_scale : 1.0f / std::sqrt(static_cast<float>(u.D));
+  p->packed = u.cu_seqlens_q != nullptr || u.cu_seqlens_k != nullptr;
+  if (p->packed) {
+    if (u.cu_seqlens_q == nullptr || u.cu_seqlens_k == nullptr) return SAGE_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(u.cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(u.cu_seqlens_k) & 3u))
+      return SAGE_ERR_INVALID_ARG;
+    if (u.total_q < 0 || u.total_k < 0) return SAGE_ERR_INVALID_ARG;
+    p->u.q_stride[0] = p->u.k_stride[0] = p->u.v_stride[0] = p->u.o_stride[0] = 0;
+  }
+  p->gs = u.gscale != SAGE_GSCALE_NONE;
+  const int64_t* strides[4] = {p->u.q_stride, p->u.k_stride, p->u.v_stride, p->u.o_stride};
+  for (const int64_t* s : strides)
+    for (int i = 0; i < 3; ++i)
+      if (s[i] < 0 || (s[i] % 8) != 0) return SAGE_ERR_INVALID_ARG;
+  p->empty = u.B == 0 || u.Hq == 0 || u.Nq == 0 || (p->packed && u.total_q == 0);
+  if (p->empty) return SAGE_OK;
+  if (u.Hkv == 0 || u.Hq % u.Hkv != 0) return SAGE_ERR_INVALID_ARG;
+  const int64_t B = u.B;
+  if (p->packed) {
+    p->rows_q = std::min<int64_t>(B * round128(u.Nq), (int64_t(u.total_q) + 127 * B) / 128 * 128);
+    p->rows_k = std::min<int64_t>(B * round128(u.Nk), (int64_t(u.total_k) + 127 * B) / 128 * 128);
+  } else {
+    p->rows_q = B * round128(u.Nq);
+    p->rows_k = B * round128(u.Nk);
+  }
+  p->rows_k = std::max<int64_t>(p->rows_k, 128);  // the K / V^T maps need one tile even with no keys
+  p->tiles_q = static_cast<int>(round128(u.Nq) / 128);
+  p->tiles_k = static_cast<int>(round128(u.Nk) / 128);
+  p->nsplit = static_cast<int>((std::max<int64_t>(u.Nq, u.Nk) + 511) / 512);
+  // Grid limits and 32-bit TMA coordinates / row indices.
+  const int64_t lim = int64_t(1) << 31;
+  if (u.B > 65535 || u.Hq > 65535) return SAGE_ERR_UNSUPPORTED;
+  if (int64_t(u.Hq) * p->rows_q >= lim || int64_t(u.Hkv) * p->rows_k >= lim ||
+      int64_t(u.Hkv) * p->rows_k / 128 * u.D >= lim || 3 * int64_t(std::max(p->tiles_q, p->tiles_k)) >= lim)
+    return SAGE_ERR_UNSUPPORTED;
+  if (p->packed && (int64_t(u.total_q) + 127 * B >= lim || int64_t(u.total_k) + 127 * B >= lim))
     return SAGE_ERR_UNSUPPORTED;
   return SAGE_OK;
 }
 
-sage_fp4_sizes_t sizes_of(const Shape& s) {
-  sage_fp4_sizes_t z;
-  if (s.empty) {
-    std::memset(&z, 0, sizeof(z));
-    return z;
-  }
-  z.q_fp4 = z.k_fp4 = static_cast<size_t>(s.BH * s.Np * s.D / 2);
-  z.q_sf = z.k_sf = static_cast<size_t>(s.BH * s.Np * s.D / 16);
-  z.vt_fp4 = static_cast<size_t>(s.BH * s.D * s.Np / 2);
-  z.vt_sf = static_cast<size_t>(s.BH * (s.Np / 128) * 1024);
-  z.k_mean = static_cast<size_t>(s.BH * s.D * 4);
+sage_fp4_problem_sizes_t sizes_of(const Prob& p) {
+  sage_fp4_problem_sizes_t z;
+  std::memset(&z, 0, sizeof(z));
+  if (p.empty) return z;
+  const int64_t D = p.u.D, B = p.u.B, Hq = p.u.Hq, Hkv = p.u.Hkv;
+  z.q_fp4 = static_cast<size_t>(Hq * p.rows_q * D / 2);
+  z.q_sf = static_cast<size_t>(Hq * p.rows_q * D / 16);
+  z.k_fp4 = static_cast<size_t>(Hkv * p.rows_k * D / 2);
+  z.k_sf = static_cast<size_t>(Hkv * p.rows_k * D / 16);
+  z.vt_fp4 = static_cast<size_t>(Hkv * p.rows_k * D / 2);
+  z.vt_sf = static_cast<size_t>(Hkv * p.rows_k / 128 * 1024);
+  z.k_mean = static_cast<size_t>(B * Hkv * D * 4);
+  z.amax = static_cast<size_t>(3 * B * Hq * 4);
+  z.seq = p.packed ? static_cast<size_t>((2 * (B + 1) + 4) * 4) : 0;
+  const int64_t ns = p.nsplit;
+  size_t scratch = 0;
+  if (p.u.smooth_k || p.gs) scratch += up256(static_cast<size_t>(B * Hkv * ns * D * 8));
+  if (p.gs)
+    scratch += 2 * up256(static_cast<size_t>(B * Hkv * ns * D * 4)) + up256(static_cast<size_t>(B * Hq * ns * 4)) +
+               up256(static_cast<size_t>(B * Hkv * ns * 4));
+  z.scratch = scratch;
+  z.workspace = up256(z.q_fp4) + up256(z.q_sf) + up256(z.k_fp4) + up256(z.k_sf) + up256(z.vt_fp4) +
+                up256(z.vt_sf) + up256(z.k_mean) + up256(z.amax) + up256(z.seq) + z.scratch;
   return z;
 }
 
-size_t scratch_of(const Shape& s) {
-  return s.empty ? 0 : static_cast<size_t>(s.BH * s.nsplit * s.D * 8);
-}
-
-size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
-
-struct Carved {
-  uint8_t *q_fp4, *q_sf, *k_fp4, *k_sf, *vt_fp4, *vt_sf;
-  float* k_mean;
-  void* scratch;
-  size_t total;
-};
-
-Carved carve(const Shape& s, void* base) {
-  const sage_fp4_sizes_t z = sizes_of(s);
-  uint8_t* p = static_cast<uint8_t*>(base);
+// Carve a workspace (256-byte aligned) into the quantized bundle followed by the scratch.
+void carve(const Prob& p, void* base, sage_fp4_quantized_t* qz, void** scratch) {
+  const sage_fp4_problem_sizes_t z = sizes_of(p);
+  uint8_t* b = static_cast<uint8_t*>(base);
   size_t off = 0;
-  Carved c;
-  auto take = [&](size_t n) { uint8_t* r = p ? p + off : nullptr; off += up256(n); return r; };
-  c.q_fp4 = take(z.q_fp4);
-  c.q_sf = take(z.q_sf);
-  c.k_fp4 = take(z.k_fp4);
-  c.k_sf = take(z.k_sf);
-  c.vt_fp4 = take(z.vt_fp4);
-  c.vt_sf = take(z.vt_sf);
-  c.k_mean = reinterpret_cast<float*>(take(z.k_mean));
-  c.scratch = take(scratch_of(s));
-  c.total = off;
-  return c;
+  auto take = [&](size_t n) { uint8_t* r = b + off; off += up256(n); return r; };
+  qz->q_fp4 = take(z.q_fp4);
+  qz->q_sf = take(z.q_sf);
+  qz->k_fp4 = take(z.k_fp4);
+  qz->k_sf = take(z.k_sf);
+  qz->vt_fp4 = take(z.vt_fp4);
+  qz->vt_sf = take(z.vt_sf);
+  qz->k_mean = reinterpret_cast<float*>(take(z.k_mean));
+  qz->amax = reinterpret_cast<float*>(take(z.amax));
+  qz->seq = p.packed ? reinterpret_cast<int32_t*>(take(z.seq)) : nullptr;
+  *scratch = z.scratch ? b + off : nullptr;
 }
 
-sage_status_t run_quantize(const Shape& s, const void* q, const void* k, const void* v, int dtype,
-                           int smooth_k, uint8_t* q_fp4, uint8_t* q_sf, uint8_t* k_fp4, uint8_t* k_sf,
-                           uint8_t* vt_fp4, uint8_t* vt_sf, float* k_mean, void* scratch,
-                           cudaStream_t stream) {
-  sage::QuantParams p;
-  p.q = q;
-  p.k = k;
-  p.v = v;
-  p.dtype = dtype;
-  p.BH = static_cast<int>(s.BH);
-  p.N = static_cast<int>(s.N);
-  p.Np = static_cast<int>(s.Np);
-  p.D = static_cast<int>(s.D);
-  p.smooth_k = smooth_k ? 1 : 0;
-  p.nsplit = static_cast<int>(s.nsplit);
-  p.q_fp4 = q_fp4;
-  p.q_sf = q_sf;
-  p.k_fp4 = k_fp4;
-  p.k_sf = k_sf;
-  p.vt_fp4 = vt_fp4;
-  p.vt_sf = vt_sf;
-  p.k_mean = k_mean;
-  p.partial = static_cast<double*>(scratch);
-  return cuda_status(sage::launch_quantize(p, stream));
+sage::SeqMap seq_map(const Prob& p, const sage_fp4_quantized_t& qz) {
+  sage::SeqMap m;
+  m.Nq = p.u.Nq;
+  m.Nk = p.u.Nk;
+  if (p.packed) {
+    m.cu_q = p.u.cu_seqlens_q;
+    m.cu_k = p.u.cu_seqlens_k;
+    m.pad_q = qz.seq;
+    m.pad_k = qz.seq + (p.u.B + 1);
+    m.bad = reinterpret_cast<const uint32_t*>(qz.seq + 2 * (p.u.B + 1));
+  } else {
+    m.cu_q = m.cu_k = m.pad_q = m.pad_k = nullptr;
+    m.bad = nullptr;
+  }
+  return m;
 }
 
-sage_status_t build_maps(const Shape& s, const uint8_t* q_fp4, const uint8_t* k_fp4,
-                         const uint8_t* vt_fp4, sage::TensorMaps* m) {
-  const uint64_t inner = static_cast<uint64_t>(s.D / 2);
-  const CUtensorMapSwizzle swqk = s.D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+sage::Strides strides_of(const int64_t s[3]) { return sage::Strides{s[0], s[1], s[2]}; }
+
+sage_status_t check_bundle(const Prob& p, const sage_fp4_quantized_t* qz, bool need_kmean) {
+  if (qz == nullptr) return SAGE_ERR_INVALID_ARG;
+  const void* ptrs[] = {qz->q_fp4, qz->q_sf, qz->k_fp4, qz->k_sf, qz->vt_fp4, qz->vt_sf};
+  for (const void* ptr : ptrs)
+    if (ptr == nullptr || !aligned16(ptr)) return SAGE_ERR_INVALID_ARG;
+  if (need_kmean && (qz->k_mean == nullptr || !aligned16(qz->k_mean))) return SAGE_ERR_INVALID_ARG;
+  if (p.gs && (qz->amax == nullptr || !aligned16(qz->amax))) return SAGE_ERR_INVALID_ARG;
+  if (p.packed && (qz->seq == nullptr || !aligned16(qz->seq))) return SAGE_ERR_INVALID_ARG;
+  return SAGE_OK;
+}
+
+sage_status_t run_quantize(const Prob& p, const void* q, const void* k, const void* v,
+                           const sage_fp4_quantized_t& qz, void* scratch, cudaStream_t stream) {
+  uint32_t* err = nullptr;
+  if (sage_status_t st = error_word(&err); st != SAGE_OK) return st;
+  sage::QuantParams k_;
+  std::memset(&k_, 0, sizeof(k_));
+  k_.q = q;
+  k_.k = k;
+  k_.v = v;
+  k_.sq = strides_of(p.u.q_stride);
+  k_.sk = strides_of(p.u.k_stride);
+  k_.sv = strides_of(p.u.v_stride);
+  k_.dtype = p.u.dtype;
+  k_.B = p.u.B;
+  k_.Hq = p.u.Hq;
+  k_.Hkv = p.u.Hkv;
+  k_.D = p.u.D;
+  k_.seq = seq_map(p, qz);
+  k_.smooth_k = p.u.smooth_k ? 1 : 0;
+  k_.gscale = p.u.gscale;
+  k_.nsplit = p.nsplit;
+  k_.amax_stride = p.u.B * p.u.Hq;
+  k_.q_fp4 = qz.q_fp4;
+  k_.q_sf = qz.q_sf;
+  k_.k_fp4 = qz.k_fp4;
+  k_.k_sf = qz.k_sf;
+  k_.vt_fp4 = qz.vt_fp4;
+  k_.vt_sf = qz.vt_sf;
+  k_.k_mean = qz.k_mean;
+  k_.amax = qz.amax;
+  const int64_t B = p.u.B, Hq = p.u.Hq, Hkv = p.u.Hkv, ns = p.nsplit, D = p.u.D;
+  uint8_t* s = static_cast<uint8_t*>(scratch);
+  auto take = [&](size_t n) { uint8_t* r = s; s += up256(n); return r; };
+  if (p.u.smooth_k || p.gs) k_.ksum = reinterpret_cast<double*>(take(static_cast<size_t>(B * Hkv * ns * D * 8)));
+  if (p.gs) {
+    k_.kmax = reinterpret_cast<float*>(take(static_cast<size_t>(B * Hkv * ns * D * 4)));
+    k_.kmin = reinterpret_cast<float*>(take(static_cast<size_t>(B * Hkv * ns * D * 4)));
+    k_.qamax = reinterpret_cast<float*>(take(static_cast<size_t>(B * Hq * ns * 4)));
+    k_.vamax = reinterpret_cast<float*>(take(static_cast<size_t>(B * Hkv * ns * 4)));
+  }
+  if (p.packed) {
+    k_.total_q = p.u.total_q;
+    k_.total_k = p.u.total_k;
+    k_.pad_q_out = qz.seq;
+    k_.pad_k_out = qz.seq + (p.u.B + 1);
+    k_.bad_out = reinterpret_cast<uint32_t*>(qz.seq + 2 * (p.u.B + 1));
+  }
+  k_.err = err;
+  return cuda_status(sage::launch_quantize(k_, sage::QuantLaunch{p.tiles_q, p.tiles_k}, stream));
+}
+
+sage_status_t build_maps(const Prob& p, const uint8_t* q_fp4, const uint8_t* k_fp4, const uint8_t* vt_fp4,
+                         sage::TensorMaps* m) {
+  const uint64_t inner = static_cast<uint64_t>(p.u.D / 2);
+  const CUtensorMapSwizzle swqk = p.u.D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
   sage_status_t st;
-  if ((st = make_map(&m->q, q_fp4, inner, s.BH * s.Np, static_cast<uint32_t>(inner), 128, swqk)) != SAGE_OK) return st;
-  if ((st = make_map(&m->k, k_fp4, inner, s.BH * s.Np, static_cast<uint32_t>(inner), 128, swqk)) != SAGE_OK) return st;
+  if ((st = make_map(&m->q, q_fp4, inner, p.u.Hq * p.rows_q, static_cast<uint32_t>(inner), 128, swqk)) != SAGE_OK) return st;
+  if ((st = make_map(&m->k, k_fp4, inner, p.u.Hkv * p.rows_k, static_cast<uint32_t>(inner), 128, swqk)) != SAGE_OK) return st;
   if (vt_fp4 != nullptr &&
-      (st = make_map(&m->v, vt_fp4, s.Np / 2, s.BH * s.D, 64, static_cast<uint32_t>(s.D), CU_TENSOR_MAP_SWIZZLE_64B)) != SAGE_OK)
+      (st = make_map(&m->v, vt_fp4, 64, p.u.Hkv * p.rows_k / 128 * p.u.D, 64, static_cast<uint32_t>(p.u.D),
+                     CU_TENSOR_MAP_SWIZZLE_64B)) != SAGE_OK)
     return st;
   return SAGE_OK;
 }
 
-sage_status_t fill_attn_params(const Shape& s, float sm_scale, int causal, sage::AttnParams* p) {
+sage_status_t base_params(int D, float sm_scale, int causal, sage::AttnParams* a) {
+  std::memset(a, 0, sizeof(*a));
   uint32_t* err = nullptr;
   if (sage_status_t st = error_word(&err); st != SAGE_OK) return st;
-  const float scale = sm_scale > 0.0f ? sm_scale : 1.0f / std::sqrt(static_cast<float>(s.D));
-  p->BH = static_cast<int>(s.BH);
-  p->N = static_cast<int>(s.N);
-  p->Np = static_cast<int>(s.Np);
-  p->D = static_cast<int>(s.D);
-  p->causal = causal ? 1 : 0;
-  p->sm_scale = scale;
-  p->sm_scale_log2 = scale * 1.4426950408889634f;
-  p->err = err;
-  p->timeout_ns = g_timeout_ns.load();
-  p->debug_flags = g_debug_flags.load();
+  a->D = D;
+  a->causal = causal ? 1 : 0;
+  a->sm_scale = sm_scale;
+  a->sm_scale_log2 = sm_scale * 1.4426950408889634f;
+  a->err = err;
+  a->timeout_ns = g_timeout_ns.load();
+  a->debug_flags = g_debug_flags.load();
   return SAGE_OK;
 }
 
-sage_status_t run_attention(const Shape& s, const uint8_t* q_fp4, const uint8_t* q_sf,
-                            const uint8_t* k_fp4, const uint8_t* k_sf, const uint8_t* vt_fp4,
-                            const uint8_t* vt_sf, void* out, int out_dtype, int causal,
-                            float sm_scale, cudaStream_t stream) {
+sage_status_t run_attention(const Prob& p, const sage_fp4_quantized_t& qz, void* out, cudaStream_t stream) {
   sage::TensorMaps m;
-  if (sage_status_t st = build_maps(s, q_fp4, k_fp4, vt_fp4, &m); st != SAGE_OK) return st;
-  sage::AttnParams p;
-  if (sage_status_t st = fill_attn_params(s, sm_scale, causal, &p); st != SAGE_OK) return st;
-  p.q_sf = q_sf;
-  p.k_sf = k_sf;
-  p.vt_sf = vt_sf;
-  p.out = out;
-  p.out_dtype = out_dtype;
-  return cuda_status(sage::launch_attention(m, p, stream));
+  if (sage_status_t st = build_maps(p, qz.q_fp4, qz.k_fp4, qz.vt_fp4, &m); st != SAGE_OK) return st;
+  sage::AttnParams a;
+  if (sage_status_t st = base_params(p.u.D, p.u.sm_scale, p.u.causal, &a); st != SAGE_OK) return st;
+  a.q_sf = qz.q_sf;
+  a.k_sf = qz.k_sf;
+  a.vt_sf = qz.vt_sf;
+  a.out = out;
+  a.so = strides_of(p.u.o_stride);
+  a.out_dtype = p.u.dtype;
+  a.B = p.u.B;
+  a.Hq = p.u.Hq;
+  a.Hkv = p.u.Hkv;
+  a.group = p.u.Hq / p.u.Hkv;
+  a.seq = seq_map(p, qz);
+  a.amax = p.gs ? qz.amax : nullptr;
+  a.gscale = p.u.gscale;
+  a.amax_stride = p.u.B * p.u.Hq;
+  return cuda_status(sage::launch_attention(m, a, p.tiles_q, stream));
 }
 
-bool valid_dtype(sage_dtype_t d) { return d == SAGE_BF16 || d == SAGE_F16; }
+// The dense [B, H, N, D] contiguous problem of the original entry points.
+sage_fp4_problem_t dense_problem(int B, int H, int N, int D, int dtype, int causal, float sm_scale, int smooth_k) {
+  sage_fp4_problem_t u;
+  std::memset(&u, 0, sizeof(u));
+  u.B = B;
+  u.Hq = u.Hkv = H;
+  u.D = D;
+  u.Nq = u.Nk = N;
+  const int64_t s[3] = {int64_t(H) * N * D, int64_t(N) * D, D};
+  for (int i = 0; i < 3; ++i) u.q_stride[i] = u.k_stride[i] = u.v_stride[i] = u.o_stride[i] = s[i];
+  u.dtype = static_cast<sage_dtype_t>(dtype);
+  u.causal = causal;
+  u.sm_scale = sm_scale;
+  u.smooth_k = smooth_k;
+  u.gscale = SAGE_GSCALE_NONE;
+  return u;
+}
 
 }  // namespace
 
@@ -240,24 +355,90 @@ const char* sage_status_string(sage_status_t status) {
   return "SAGE_ERR_UNKNOWN";
 }
 
+// ------------------------------------------------------------ general problem ----
+
+sage_status_t sage_fp4_problem_sizes(const sage_fp4_problem_t* problem, sage_fp4_problem_sizes_t* sizes) {
+  if (sizes == nullptr) return SAGE_ERR_INVALID_ARG;
+  Prob p;
+  if (sage_status_t st = check_problem(problem, &p); st != SAGE_OK) return st;
+  *sizes = sizes_of(p);
+  return SAGE_OK;
+}
+
+sage_status_t sage_fp4_quantize(const sage_fp4_problem_t* problem, const void* q, const void* k,
+                                const void* v, const sage_fp4_quantized_t* qz, void* scratch,
+                                size_t scratch_bytes, void* stream) {
+  Prob p;
+  if (sage_status_t st = check_problem(problem, &p); st != SAGE_OK) return st;
+  if (p.empty) return SAGE_OK;
+  const void* ptrs[] = {q, k, v};
+  for (const void* ptr : ptrs)
+    if (ptr == nullptr || !aligned16(ptr)) return SAGE_ERR_INVALID_ARG;
+  if (sage_status_t st = check_bundle(p, qz, true); st != SAGE_OK) return st;
+  const size_t need = sizes_of(p).scratch;
+  if (need > 0 && (scratch == nullptr || !aligned16(scratch) || scratch_bytes < need)) return SAGE_ERR_INVALID_ARG;
+  return run_quantize(p, q, k, v, *qz, scratch, static_cast<cudaStream_t>(stream));
+}
+
+sage_status_t sage_fp4_attn_quantized(const sage_fp4_problem_t* problem, const sage_fp4_quantized_t* qz,
+                                      void* out, void* stream) {
+  Prob p;
+  if (sage_status_t st = check_problem(problem, &p); st != SAGE_OK) return st;
+  if (p.empty) return SAGE_OK;
+  if (out == nullptr || !aligned16(out)) return SAGE_ERR_INVALID_ARG;
+  if (sage_status_t st = check_bundle(p, qz, false); st != SAGE_OK) return st;
+  return run_attention(p, *qz, out, static_cast<cudaStream_t>(stream));
+}
+
+sage_status_t sage_fp4_attn(const sage_fp4_problem_t* problem, const void* q, const void* k, const void* v,
+                            void* out, void* workspace, size_t ws_bytes, void* stream) {
+  Prob p;
+  if (sage_status_t st = check_problem(problem, &p); st != SAGE_OK) return st;
+  if (p.empty) return SAGE_OK;
+  const void* ptrs[] = {q, k, v, out};
+  for (const void* ptr : ptrs)
+    if (ptr == nullptr || !aligned16(ptr)) return SAGE_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SAGE_ERR_INVALID_ARG;
+  if (ws_bytes < sizes_of(p).workspace) return SAGE_ERR_INVALID_ARG;
+  sage_fp4_quantized_t qz;
+  void* scratch = nullptr;
+  carve(p, workspace, &qz, &scratch);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (sage_status_t r = run_quantize(p, q, k, v, qz, scratch, st); r != SAGE_OK) return r;
+  return run_attention(p, qz, out, st);
+}
+
+// ------------------------------------------------- dense [B, H, N, D] problems ----
+
 sage_status_t sage_fp4_quantized_sizes(int B, int H, int N, int D, sage_fp4_sizes_t* sizes) {
   if (sizes == nullptr) return SAGE_ERR_INVALID_ARG;
-  Shape s;
-  if (sage_status_t st = check_shape(B, H, N, D, &s); st != SAGE_OK) return st;
-  *sizes = sizes_of(s);
+  const sage_fp4_problem_t u = dense_problem(B, H, N, D, SAGE_BF16, 0, 0.0f, 1);
+  Prob p;
+  if (sage_status_t st = check_problem(&u, &p); st != SAGE_OK) return st;
+  const sage_fp4_problem_sizes_t z = sizes_of(p);
+  sizes->q_fp4 = z.q_fp4;
+  sizes->q_sf = z.q_sf;
+  sizes->k_fp4 = z.k_fp4;
+  sizes->k_sf = z.k_sf;
+  sizes->vt_fp4 = z.vt_fp4;
+  sizes->vt_sf = z.vt_sf;
+  sizes->k_mean = z.k_mean;
   return SAGE_OK;
 }
 
 size_t sage_fp4_quantize_scratch_bytes(int B, int H, int N, int D) {
-  Shape s;
-  if (check_shape(B, H, N, D, &s) != SAGE_OK) return 0;
-  return scratch_of(s);
+  const sage_fp4_problem_t u = dense_problem(B, H, N, D, SAGE_BF16, 0, 0.0f, 1);
+  Prob p;
+  if (check_problem(&u, &p) != SAGE_OK || p.empty) return 0;
+  // The binary64 partial sums, then room for the K mean when the caller passes none.
+  return sizes_of(p).scratch + up256(sizes_of(p).k_mean);
 }
 
 size_t sage_fp4_workspace_bytes(int B, int H, int N, int D) {
-  Shape s;
-  if (check_shape(B, H, N, D, &s) != SAGE_OK || s.empty) return 0;
-  return carve(s, nullptr).total;
+  const sage_fp4_problem_t u = dense_problem(B, H, N, D, SAGE_BF16, 0, 0.0f, 1);
+  Prob p;
+  if (check_problem(&u, &p) != SAGE_OK || p.empty) return 0;
+  return sizes_of(p).workspace;
 }
 
 sage_status_t sage_fp4_quantize_qkv(const void* q, const void* k, const void* v, sage_dtype_t dtype,
@@ -265,19 +446,30 @@ sage_status_t sage_fp4_quantize_qkv(const void* q, const void* k, const void* v,
                                     uint8_t* q_sf, uint8_t* k_fp4, uint8_t* k_sf, uint8_t* vt_fp4,
                                     uint8_t* vt_sf, float* k_mean, void* scratch,
                                     size_t scratch_bytes, void* stream) {
-  Shape s;
-  if (sage_status_t st = check_shape(B, H, N, D, &s); st != SAGE_OK) return st;
   if (!valid_dtype(dtype)) return SAGE_ERR_INVALID_ARG;
-  if (s.empty) return SAGE_OK;
-  const void* ptrs[] = {q, k, v, q_fp4, q_sf, k_fp4, k_sf, vt_fp4, vt_sf};
+  const sage_fp4_problem_t u = dense_problem(B, H, N, D, dtype, 0, 0.0f, smooth_k ? 1 : 0);
+  Prob p;
+  if (sage_status_t st = check_problem(&u, &p); st != SAGE_OK) return st;
+  if (p.empty) return SAGE_OK;
+  const void* ptrs[] = {q, k, v};
   for (const void* ptr : ptrs)
     if (ptr == nullptr || !aligned16(ptr)) return SAGE_ERR_INVALID_ARG;
-  if (smooth_k) {
-    if (scratch == nullptr || !aligned16(scratch) || scratch_bytes < scratch_of(s)) return SAGE_ERR_INVALID_ARG;
-    if (k_mean != nullptr && !aligned16(k_mean)) return SAGE_ERR_INVALID_ARG;
-  }
-  return run_quantize(s, q, k, v, dtype, smooth_k, q_fp4, q_sf, k_fp4, k_sf, vt_fp4, vt_sf, k_mean,
-                      scratch, static_cast<cudaStream_t>(stream));
+  sage_fp4_quantized_t qz;
+  std::memset(&qz, 0, sizeof(qz));
+  qz.q_fp4 = q_fp4;
+  qz.q_sf = q_sf;
+  qz.k_fp4 = k_fp4;
+  qz.k_sf = k_sf;
+  qz.vt_fp4 = vt_fp4;
+  qz.vt_sf = vt_sf;
+  qz.k_mean = k_mean;
+  if (sage_status_t st = check_bundle(p, &qz, false); st != SAGE_OK) return st;
+  if (k_mean != nullptr && !aligned16(k_mean)) return SAGE_ERR_INVALID_ARG;
+  const sage_fp4_problem_sizes_t z = sizes_of(p);
+  const size_t need = smooth_k ? z.scratch + (k_mean ? 0 : up256(z.k_mean)) : 0;
+  if (need > 0 && (scratch == nullptr || !aligned16(scratch) || scratch_bytes < need)) return SAGE_ERR_INVALID_ARG;
+  if (smooth_k && k_mean == nullptr) qz.k_mean = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + z.scratch);
+  return run_quantize(p, q, k, v, qz, smooth_k ? scratch : nullptr, static_cast<cudaStream_t>(stream));
 }
 
 sage_status_t sage_fp4_attn_fwd_quantized(const uint8_t* q_fp4, const uint8_t* q_sf,
@@ -285,55 +477,39 @@ sage_status_t sage_fp4_attn_fwd_quantized(const uint8_t* q_fp4, const uint8_t* q
                                           const uint8_t* vt_fp4, const uint8_t* vt_sf, void* out,
                                           sage_dtype_t out_dtype, int B, int H, int N, int D,
                                           int causal, float sm_scale, void* stream) {
-  Shape s;
-  if (sage_status_t st = check_shape(B, H, N, D, &s); st != SAGE_OK) return st;
-  if (!valid_dtype(out_dtype)) return SAGE_ERR_INVALID_ARG;
-  if (s.empty) return SAGE_OK;
-  const void* ptrs[] = {q_fp4, q_sf, k_fp4, k_sf, vt_fp4, vt_sf, out};
-  for (const void* ptr : ptrs)
-    if (ptr == nullptr || !aligned16(ptr)) return SAGE_ERR_INVALID_ARG;
-  if (!std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
-  return run_attention(s, q_fp4, q_sf, k_fp4, k_sf, vt_fp4, vt_sf, out, out_dtype, causal, sm_scale,
-                       static_cast<cudaStream_t>(stream));
+  const sage_fp4_problem_t u = dense_problem(B, H, N, D, out_dtype, causal, sm_scale, 1);
+  sage_fp4_quantized_t qz;
+  std::memset(&qz, 0, sizeof(qz));
+  qz.q_fp4 = const_cast<uint8_t*>(q_fp4);
+  qz.q_sf = const_cast<uint8_t*>(q_sf);
+  qz.k_fp4 = const_cast<uint8_t*>(k_fp4);
+  qz.k_sf = const_cast<uint8_t*>(k_sf);
+  qz.vt_fp4 = const_cast<uint8_t*>(vt_fp4);
+  qz.vt_sf = const_cast<uint8_t*>(vt_sf);
+  return sage_fp4_attn_quantized(&u, &qz, out, stream);
 }
 
 sage_status_t sage_fp4_attn_fwd_ex(const void* q, const void* k, const void* v, void* out,
                                    sage_dtype_t dtype, int B, int H, int N, int D, int causal,
                                    float sm_scale, void* workspace, size_t ws_bytes, void* stream) {
-  Shape s;
-  if (sage_status_t st = check_shape(B, H, N, D, &s); st != SAGE_OK) return st;
-  if (!valid_dtype(dtype)) return SAGE_ERR_INVALID_ARG;
-  if (s.empty) return SAGE_OK;
-  const void* ptrs[] = {q, k, v, out};
-  for (const void* ptr : ptrs)
-    if (ptr == nullptr || !aligned16(ptr)) return SAGE_ERR_INVALID_ARG;
-  if (!std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
-  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SAGE_ERR_INVALID_ARG;
-  Carved c = carve(s, workspace);
-  if (ws_bytes < c.total) return SAGE_ERR_INVALID_ARG;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  sage_status_t r = run_quantize(s, q, k, v, dtype, 1, c.q_fp4, c.q_sf, c.k_fp4, c.k_sf, c.vt_fp4,
-                                 c.vt_sf, c.k_mean, c.scratch, st);
-  if (r != SAGE_OK) return r;
-  return run_attention(s, c.q_fp4, c.q_sf, c.k_fp4, c.k_sf, c.vt_fp4, c.vt_sf, out, dtype, causal,
-                       sm_scale, st);
+  const sage_fp4_problem_t u = dense_problem(B, H, N, D, dtype, causal, sm_scale, 1);
+  return sage_fp4_attn(&u, q, k, v, out, workspace, ws_bytes, stream);
 }
 
 sage_status_t sage_fp4_attn_fwd(const void* q, const void* k, const void* v, void* out, int B,
                                 int H, int N, int D, int causal, float sm_scale, void* stream) {
-  Shape s;
-  if (sage_status_t st = check_shape(B, H, N, D, &s); st != SAGE_OK) return st;
-  if (s.empty) return SAGE_OK;
+  const sage_fp4_problem_t u = dense_problem(B, H, N, D, SAGE_BF16, causal, sm_scale, 1);
+  Prob p;
+  if (sage_status_t st = check_problem(&u, &p); st != SAGE_OK) return st;
+  if (p.empty) return SAGE_OK;
   const void* ptrs[] = {q, k, v, out};
   for (const void* ptr : ptrs)
     if (ptr == nullptr || !aligned16(ptr)) return SAGE_ERR_INVALID_ARG;
-  if (!std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t bytes = carve(s, nullptr).total;
+  const size_t bytes = sizes_of(p).workspace;
   void* ws = nullptr;
   if (cudaMallocAsync(&ws, bytes, st) != cudaSuccess) return SAGE_ERR_CUDA;
-  sage_status_t r = sage_fp4_attn_fwd_ex(q, k, v, out, SAGE_BF16, B, H, N, D, causal, sm_scale, ws,
-                                         bytes, stream);
+  sage_status_t r = sage_fp4_attn(&u, q, k, v, out, ws, bytes, stream);
   const cudaError_t e = cudaFreeAsync(ws, st);
   if (r == SAGE_OK && e != cudaSuccess) r = SAGE_ERR_CUDA;
   return r;
@@ -342,24 +518,24 @@ sage_status_t sage_fp4_attn_fwd(const void* q, const void* k, const void* v, voi
 sage_status_t sage_fp4_qk_scores(const uint8_t* q_fp4, const uint8_t* q_sf, const uint8_t* k_fp4,
                                  const uint8_t* k_sf, float* s_out, int B, int H, int N, int D,
                                  float sm_scale, void* stream) {
-  Shape s;
-  if (sage_status_t st = check_shape(B, H, N, D, &s); st != SAGE_OK) return st;
-  if (s.empty) return SAGE_OK;
+  const sage_fp4_problem_t u = dense_problem(B, H, N, D, SAGE_BF16, 0, sm_scale, 1);
+  Prob p;
+  if (sage_status_t st = check_problem(&u, &p); st != SAGE_OK) return st;
+  if (p.empty) return SAGE_OK;
   const void* ptrs[] = {q_fp4, q_sf, k_fp4, k_sf, s_out};
   for (const void* ptr : ptrs)
     if (ptr == nullptr || !aligned16(ptr)) return SAGE_ERR_INVALID_ARG;
-  if (!std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
-  if (s.Np / 128 > 65535) return SAGE_ERR_UNSUPPORTED;
+  if (p.tiles_q > 65535) return SAGE_ERR_UNSUPPORTED;
   sage::TensorMaps m;
-  if (sage_status_t st = build_maps(s, q_fp4, k_fp4, nullptr, &m); st != SAGE_OK) return st;
-  sage::AttnParams p;
-  if (sage_status_t st = fill_attn_params(s, sm_scale, 0, &p); st != SAGE_OK) return st;
-  p.q_sf = q_sf;
-  p.k_sf = k_sf;
-  p.vt_sf = nullptr;
-  p.out = s_out;
-  p.out_dtype = 0;
-  return cuda_status(sage::launch_qk_scores(m, p, static_cast<cudaStream_t>(stream)));
+  if (sage_status_t st = build_maps(p, q_fp4, k_fp4, nullptr, &m); st != SAGE_OK) return st;
+  sage::AttnParams a;
+  if (sage_status_t st = base_params(D, p.u.sm_scale, 0, &a); st != SAGE_OK) return st;
+  a.q_sf = q_sf;
+  a.k_sf = k_sf;
+  a.out = s_out;
+  a.BH = B * H;
+  a.Np = static_cast<int>(round128(N));
+  return cuda_status(sage::launch_qk_scores(m, a, static_cast<cudaStream_t>(stream)));
 }
 
 sage_status_t sage_fp4_get_device_error(uint32_t* word, void* stream) {
@@ -372,7 +548,8 @@ sage_status_t sage_fp4_get_device_error(uint32_t* word, void* stream) {
   if (cudaMemsetAsync(dev, 0, sizeof(uint32_t), s) != cudaSuccess) return SAGE_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return SAGE_ERR_CUDA;
   *word = host;
-  return host == 0 ? SAGE_OK : SAGE_ERR_TIMEOUT;
+  if (host == 0) return SAGE_OK;
+  return (host & sage::kDevErrTimeout) ? SAGE_ERR_TIMEOUT : SAGE_ERR_INVALID_ARG;
 }
 
 const char* sage_fp4_last_cuda_error(void) { return g_last_error; }

@@ -11,33 +11,122 @@ namespace sage {
 enum : int { kDtypeBF16 = 0, kDtypeF16 = 1 };
 
 // Bits of the device error word.
-enum : uint32_t { kDevErrTimeout = 1u };
+enum : uint32_t { kDevErrTimeout = 1u, kDevErrSeqlens = 2u };
 
+// Second-level scale modes (one FP32 factor per tensor or per (sequence, head)).
+enum : int { kGscaleNone = 0, kGscaleTensor = 1, kGscaleHead = 2 };
+
+// 448 * 6: E4M3 max times E2M1 max, the target of every two-level scaling.
+constexpr float kTwoLevelTarget = 2688.0f;
+
+// Element strides of (sequence, head, token); channels are contiguous.
+struct Strides {
+  int64_t b, h, n;
+};
+
+// Where each sequence lives. Dense problems (cu_q == nullptr): B sequences of Nq queries
+// and Nk keys, sequence b starting at token 0 of batch b. Packed problems: sequence b
+// holds tokens cu_q[b] .. cu_q[b+1] of the packed tensors; pad_q[b] is the number of
+// padded (multiple-of-128) query tokens of the sequences before it, computed on the
+// device; *bad != 0 when the sequence table failed validation (kernels then do nothing).
+struct SeqMap {
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  const int32_t* pad_q;
+  const int32_t* pad_k;
+  const uint32_t* bad;
+  int Nq, Nk;
+};
+
+struct SeqInfo {
+  int len_q, len_k;    // tokens
+  int tok_q, tok_k;    // first token in the (packed) input / output tensors
+  int prow_q, prow_k;  // padded tokens of all earlier sequences
+};
+
+__device__ __forceinline__ int round128(int x) { return (x + 127) & ~127; }
+
+__device__ __forceinline__ SeqInfo seq_info(const SeqMap& m, int b) {
+  SeqInfo s;
+  if (m.cu_q == nullptr) {
+    s.len_q = m.Nq;
+    s.len_k = m.Nk;
+    s.tok_q = 0;
+    s.tok_k = 0;
+    s.prow_q = b * round128(m.Nq);
+    s.prow_k = b * round128(m.Nk);
+  } else {
+    s.tok_q = m.cu_q[b];
+    s.tok_k = m.cu_k[b];
+    s.len_q = m.cu_q[b + 1] - s.tok_q;
+    s.len_k = m.cu_k[b + 1] - s.tok_k;
+    s.prow_q = m.pad_q[b];
+    s.prow_k = m.pad_k[b];
+  }
+  return s;
+}
+
+__device__ __forceinline__ bool seq_table_bad(const SeqMap& m) {
+  return m.bad != nullptr && *reinterpret_cast<const volatile uint32_t*>(m.bad) != 0u;
+}
+
+// Second-level scale from a group maximum: fp32(amax / 2688), or 1 when that is 0.
+__device__ __forceinline__ float second_level_scale(float amax) {
+  const float g = __fdiv_rn(amax, kTwoLevelTarget);
+  return g > 0.0f ? g : 1.0f;
+}
+
+// Quantized layouts: the padded-token row of (sequence b, head h, token n) of Q is
+//   Hq * prow_q + h * round128(len_q) + n
+// (K and V^T likewise with Hkv, prow_k, len_k); a 128-row tile t of those rows is
+// the scale-factor tile t and the V^T tile t.
 struct QuantParams {
   const void* q;
   const void* k;
   const void* v;
+  Strides sq, sk, sv;
   int dtype;
-  int BH, N, Np, D;
+  int B, Hq, Hkv, D;
+  SeqMap seq;
   int smooth_k;
-  int nsplit;  // number of 512-token chunks of the K mean
+  int gscale;
+  int nsplit;        // 512-token chunks of the longest sequence
+  int amax_stride;   // B * Hq: distance between the Q, K and V maxima
   uint8_t* q_fp4;
   uint8_t* q_sf;
   uint8_t* k_fp4;
   uint8_t* k_sf;
   uint8_t* vt_fp4;
   uint8_t* vt_sf;
-  float* k_mean;
-  double* partial;  // [BH, nsplit, D]
+  float* k_mean;     // [B * Hkv, D]
+  float* amax;       // [3, B * Hq]; tensor mode uses element 0 of each
+  double* ksum;      // [B * Hkv, nsplit, D]
+  float* kmax;       // [B * Hkv, nsplit, D]  (second-level scale only)
+  float* kmin;       // [B * Hkv, nsplit, D]
+  float* qamax;      // [B * Hq, nsplit]
+  float* vamax;      // [B * Hkv, nsplit]
+  // Packed problems: the plan kernel's inputs and outputs.
+  int total_q, total_k;
+  int32_t* pad_q_out;
+  int32_t* pad_k_out;
+  uint32_t* bad_out;
+  uint32_t* err;
 };
 
 struct AttnParams {
   const uint8_t* q_sf;
   const uint8_t* k_sf;
   const uint8_t* vt_sf;
-  void* out;            // [BH, N, D] (attention) or float [BH, Np, Np] (scores)
+  void* out;            // attention: element (b, h, n) at b*so.b + h*so.h + (tok_q + n)*so.n;
+                        // scores: float [BH, Np, Np]
+  Strides so;
   int out_dtype;
-  int BH, N, Np, D;
+  int B, Hq, Hkv, group, D;
+  SeqMap seq;
+  const float* amax;    // second-level maxima, or nullptr
+  int gscale;
+  int amax_stride;
+  int BH, Np;           // dense S = Q^ K^^T (scores kernel only)
   int causal;
   float sm_scale;       // scale of the dot products
   float sm_scale_log2;  // sm_scale * log2(e)
@@ -52,8 +141,12 @@ struct TensorMaps {
   CUtensorMap q, k, v;
 };
 
-cudaError_t launch_quantize(const QuantParams& p, cudaStream_t stream);
-cudaError_t launch_attention(const TensorMaps& maps, const AttnParams& p, cudaStream_t stream);
+struct QuantLaunch {
+  int tiles_q, tiles_k;  // 128-token tiles of the longest query / key sequence
+};
+
+cudaError_t launch_quantize(const QuantParams& p, const QuantLaunch& l, cudaStream_t stream);
+cudaError_t launch_attention(const TensorMaps& maps, const AttnParams& p, int tiles_q, cudaStream_t stream);
 cudaError_t launch_qk_scores(const TensorMaps& maps, const AttnParams& p, cudaStream_t stream);
 
 }  // namespace sage

@@ -19,6 +19,7 @@ machine, with or without a GPU.
 from __future__ import annotations
 
 import dataclasses
+import itertools
 import math
 from typing import List, Optional
 
@@ -113,3 +114,111 @@ def make_inputs(w: Workload, device: Optional[str] = None):
     if device is not None:
         q, k, v = q.to(device), k.to(device), v.to(device)
     return q, k, v
+
+
+# ----------------------------------------------------------- general problems --
+#
+# Recipe: one CPU generator seeded with the workload's seed draws, in this order,
+# Q [Tq, Hq, D], K [Tk, Hkv, D], V [Tk, Hkv, D] ~ N(0, 1) in float32 (Tq, Tk = the summed
+# lengths; sequence b owns the next lens[b] tokens), then one K bias per (sequence, key
+# head) ~ N(0, sigma^2) [B, Hkv, D] added to that sequence's keys. Q, K and V are then
+# multiplied by q_scale, k_scale and v_scale (to reach the one-level format's range
+# limits) and cast to the dtype. Dense workloads view the same draws as [B, H, N, D]
+# ("HND") or [B, N, H, D] ("NHD") tensors.
+
+@dataclasses.dataclass(frozen=True)
+class GeneralWorkload:
+    name: str
+    Hq: int
+    Hkv: int
+    D: int
+    lens_q: tuple
+    lens_k: tuple
+    causal: bool
+    packed: bool
+    layout: str = "HND"
+    dtype: torch.dtype = torch.bfloat16
+    seed: int = 0
+    bias_sigma: float = 2.0
+    q_scale: float = 1.0
+    k_scale: float = 1.0
+    v_scale: float = 1.0
+    gscale: str = "none"
+
+    @property
+    def B(self) -> int:
+        return len(self.lens_q)
+
+    @property
+    def sm_scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+    @property
+    def ops(self) -> float:
+        """4 * Hq * Lq * Lk * D per sequence, halved when causal (the square-problem
+        convention of the dense workloads)."""
+        o = sum(4.0 * self.Hq * lq * lk * self.D for lq, lk in zip(self.lens_q, self.lens_k))
+        return o / 2 if self.causal else o
+
+    def describe(self) -> dict:
+        return {"workload": self.name, "B": self.B, "Hq": self.Hq, "Hkv": self.Hkv, "D": self.D,
+                "lens_q": list(self.lens_q) if len(self.lens_q) <= 16 else f"{len(self.lens_q)} sequences",
+                "total_q": sum(self.lens_q), "total_k": sum(self.lens_k), "causal": self.causal,
+                "packed": self.packed, "layout": self.layout,
+                "dtype": str(self.dtype).replace("torch.", ""), "seed": self.seed,
+                "gscale": self.gscale}
+
+
+def general(name: str, Hq: int, Hkv: int, D: int, lens_q, lens_k=None, causal: bool = False,
+            packed: bool = True, **kw) -> GeneralWorkload:
+    lens_q = tuple(int(x) for x in lens_q)
+    lens_k = lens_q if lens_k is None else tuple(int(x) for x in lens_k)
+    return GeneralWorkload(name, Hq, Hkv, D, lens_q, lens_k, causal, packed, **kw)
+
+
+def length_mix(count: int, lo: int, hi: int, seed: int) -> tuple:
+    """Sequence lengths drawn uniformly from [lo, hi] by a seeded CPU generator."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return tuple(int(x) for x in torch.randint(lo, hi + 1, (count,), generator=g))
+
+
+# An LLM-serving batch: 16 packed prompts of mixed length, grouped-query heads (32 query
+# heads sharing 8 key/value heads), causal.
+LLM_VARLEN_GQA = general("llm_varlen_gqa_Hq32_Hkv8_D128_16seq", 32, 8, 128,
+                         length_mix(16, 256, 16384, seed=41), causal=True, seed=41)
+
+
+def make_general_inputs(w: GeneralWorkload, device: Optional[str] = None) -> dict:
+    """Draw the inputs of a general workload. Packed: q [Tq, Hq, D], k and v [Tk, Hkv, D]
+    plus int32 cu_seqlens_q / cu_seqlens_k; dense: [B, H, N, D] ("HND") or [B, N, H, D]
+    ("NHD") tensors (every sequence then has the same lengths)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+    Tq, Tk = sum(w.lens_q), sum(w.lens_k)
+    q = torch.randn((Tq, w.Hq, w.D), generator=g, dtype=torch.float32)
+    k = torch.randn((Tk, w.Hkv, w.D), generator=g, dtype=torch.float32)
+    v = torch.randn((Tk, w.Hkv, w.D), generator=g, dtype=torch.float32)
+    bias = torch.randn((w.B, w.Hkv, w.D), generator=g, dtype=torch.float32) * w.bias_sigma
+    cu_q = torch.tensor([0] + list(itertools.accumulate(w.lens_q)), dtype=torch.int32)
+    cu_k = torch.tensor([0] + list(itertools.accumulate(w.lens_k)), dtype=torch.int32)
+    for b in range(w.B):
+        k[cu_k[b]:cu_k[b + 1]] += bias[b]
+    q, k, v = (q * w.q_scale).to(w.dtype), (k * w.k_scale).to(w.dtype), (v * w.v_scale).to(w.dtype)
+    out = {"cu_seqlens_q": cu_q, "cu_seqlens_k": cu_k}
+    if w.packed:
+        out.update(q=q, k=k, v=v)
+    else:
+        if len(set(w.lens_q)) != 1 or len(set(w.lens_k)) != 1:
+            raise ValueError("a dense workload needs equal lengths")
+        Nq, Nk = w.lens_q[0], w.lens_k[0]
+        qd = q.reshape(w.B, Nq, w.Hq, w.D)
+        kd = k.reshape(w.B, Nk, w.Hkv, w.D)
+        vd = v.reshape(w.B, Nk, w.Hkv, w.D)
+        if w.layout == "HND":
+            qd, kd, vd = (t.permute(0, 2, 1, 3).contiguous() for t in (qd, kd, vd))
+        out.update(q=qd, k=kd, v=vd)
+    if device is not None:
+        out = {n: t.to(device) for n, t in out.items()}
+    return out
+

@@ -29,16 +29,23 @@ def vt_sf_index(BH: int, Nb: int, Np: int, D: int) -> np.ndarray:
             + (d % 32) * 16 + (d // 32) * 4 + t % 4)
 
 
+def _vt_rows(vt: np.ndarray, BH: int, Np: int, D: int) -> np.ndarray:
+    """Tile-major V^T [BH * Np/128, D, 64] -> [BH, D, Np/2]."""
+    t = vt[: BH * Np * D // 2].reshape(BH, Np // 128, D, 64)
+    return np.ascontiguousarray(t.transpose(0, 2, 1, 3).reshape(BH, D, Np // 2))
+
+
 def canonical(qz: dict) -> dict:
     """GPU quantized tensors -> oracle canonical numpy layouts (padding stripped)."""
     B, H, N, D, Np = qz["B"], qz["H"], qz["N"], qz["D"], qz["Np"]
     BH = B * H
     N16 = (N + 15) // 16 * 16
     g = {k: qz[k].cpu().numpy() for k in ("q_fp4", "q_sf", "k_fp4", "k_sf", "vt_fp4", "vt_sf")}
+    vt = _vt_rows(g["vt_fp4"], BH, Np, D)
     out = {
         "q_codes": g["q_fp4"][: BH * Np * D // 2].reshape(BH, Np, D // 2)[:, :N],
         "k_codes": g["k_fp4"][: BH * Np * D // 2].reshape(BH, Np, D // 2)[:, :N],
-        "vt_codes": g["vt_fp4"][: BH * D * Np // 2].reshape(BH, D, Np // 2)[:, :, : N16 // 2],
+        "vt_codes": vt[:, :, : N16 // 2],
         "q_sf": g["q_sf"][qk_sf_index(BH, N, Np, D)],
         "k_sf": g["k_sf"][qk_sf_index(BH, N, Np, D)],
         "vt_sf": g["vt_sf"][vt_sf_index(BH, N16 // 16, Np, D)],
@@ -49,12 +56,73 @@ def canonical(qz: dict) -> dict:
     pads = {
         "q_fp4": g["q_fp4"][: BH * Np * D // 2].reshape(BH, Np, D // 2)[:, N:],
         "k_fp4": g["k_fp4"][: BH * Np * D // 2].reshape(BH, Np, D // 2)[:, N:],
-        "vt_fp4": g["vt_fp4"][: BH * D * Np // 2].reshape(BH, D, Np // 2)[:, :, (N + 1) // 2:],
+        "vt_fp4": vt[:, :, (N + 1) // 2:],
     }
     out["pads_zero"] = all(not p.any() for p in pads.values())
     for k in ("q_codes", "k_codes", "vt_codes"):
         out[k] = np.ascontiguousarray(out[k])
     return out
+
+
+def padded_offsets(lens) -> np.ndarray:
+    """Exclusive prefix sums of the lengths rounded up to 128."""
+    r = [(int(n) + 127) // 128 * 128 for n in lens]
+    return np.concatenate([[0], np.cumsum(r)]).astype(np.int64)
+
+
+def _sf_rows(sf: np.ndarray, rows: np.ndarray, D: int) -> np.ndarray:
+    """Scale bytes of padded rows `rows` (all D/16 channel blocks) -> [len(rows), D/16]."""
+    r = rows[:, None]
+    c = np.arange(D // 16)[None, :]
+    idx = ((r // 128) * (D // 64) + (16 * c) // 64) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + c % 4
+    return sf[idx]
+
+
+def canonical_problem(qz: dict, lens_q, lens_k, Hq: int, Hkv: int, D: int) -> list:
+    """Per sequence, the GPU's quantized tensors of a general problem in the oracle's
+    canonical layouts: q_codes [Hq, Lq, D/2], q_sf [Hq, Lq, D/16], k_codes / k_sf
+    [Hkv, Lk, ...], vt_codes [Hkv, D, ceil16(Lk)/2], vt_sf [Hkv, D, ceil16(Lk)/16],
+    k_mean [Hkv, D]; plus pads_zero (the padding rows and tokens hold zeros)."""
+    g = {k: qz[k].cpu().numpy() for k in ("q_fp4", "q_sf", "k_fp4", "k_sf", "vt_fp4", "vt_sf")}
+    kmean = qz["k_mean"].cpu().numpy()
+    pq, pk = padded_offsets(lens_q), padded_offsets(lens_k)
+    res = []
+    for b, (Lq, Lk) in enumerate(zip(lens_q, lens_k)):
+        Pq, Pk = (Lq + 127) // 128 * 128, (Lk + 127) // 128 * 128
+        o = {"pads_zero": True}
+        qc, qs, kc, ks = [], [], [], []
+        for h in range(Hq):
+            r0 = Hq * pq[b] + h * Pq
+            rows = np.arange(r0, r0 + Pq)
+            blk = g["q_fp4"][r0 * (D // 2):(r0 + Pq) * (D // 2)].reshape(Pq, D // 2)
+            qc.append(blk[:Lq])
+            qs.append(_sf_rows(g["q_sf"], rows[:Lq], D))
+            o["pads_zero"] &= not blk[Lq:].any()
+        vc, vs = [], []
+        L16 = (Lk + 15) // 16 * 16
+        for h in range(Hkv):
+            r0 = Hkv * pk[b] + h * Pk
+            rows = np.arange(r0, r0 + Pk)
+            blk = g["k_fp4"][r0 * (D // 2):(r0 + Pk) * (D // 2)].reshape(Pk, D // 2)
+            kc.append(blk[:Lk])
+            ks.append(_sf_rows(g["k_sf"], rows[:Lk], D))
+            o["pads_zero"] &= not blk[Lk:].any()
+            t0 = r0 // 128
+            vt = g["vt_fp4"][t0 * D * 64:(t0 + Pk // 128) * D * 64].reshape(Pk // 128, D, 64)
+            vt = vt.transpose(1, 0, 2).reshape(D, Pk // 2)
+            vc.append(vt[:, : L16 // 2])
+            o["pads_zero"] &= not vt[:, (Lk + 1) // 2:].any()
+            u = np.arange(L16 // 16)[None, :]
+            d = np.arange(D)[:, None]
+            t = t0 + (16 * u) // 128
+            uu = u % 8
+            vs.append(g["vt_sf"][(t * 2 + uu // 4) * 512 + (d % 32) * 16 + (d // 32) * 4 + uu % 4])
+        o["q_codes"], o["q_sf"] = np.stack(qc), np.stack(qs)
+        o["k_codes"], o["k_sf"] = np.stack(kc), np.stack(ks)
+        o["vt_codes"], o["vt_sf"] = np.stack(vc), np.stack(vs)
+        o["k_mean"] = kmean[b * Hkv * D:(b + 1) * Hkv * D].reshape(Hkv, D)
+        res.append(o)
+    return res
 
 
 def heads_view(t: torch.Tensor, heads) -> np.ndarray:

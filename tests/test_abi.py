@@ -60,3 +60,56 @@ def test_host_side_argument_checks(L):
     assert L.sage_fp4_attn_fwd(None, None, None, None, 0, 4, 128, 64, 0, ctypes.c_float(0.0), None) == 0
     assert L.sage_status_string(4) == b"SAGE_ERR_TIMEOUT"
     assert sage.workspace_bytes(1, 24, 32768, 128) > 0
+
+
+def _dense_pr(sage, **kw):
+    args = dict(B=2, Hq=8, Hkv=2, D=128, Nq=300, Nk=500, dtype=__import__("torch").bfloat16,
+                q_stride=(8 * 300 * 128, 300 * 128, 128), k_stride=(2 * 500 * 128, 500 * 128, 128),
+                v_stride=(2 * 500 * 128, 500 * 128, 128), o_stride=(8 * 300 * 128, 300 * 128, 128))
+    args.update(kw)
+    return sage.make_problem(**args)
+
+
+def test_general_problem_sizes_on_host(L):
+    import microscaling_fp4_quantized_b200 as sage
+    z = sage.problem_sizes(_dense_pr(sage))
+    # padded rows: B * round128(Nq) per query head, B * round128(Nk) per key/value head
+    assert z["q_fp4"] == 8 * 2 * 384 * 64 and z["q_sf"] == 8 * 2 * 384 * 8
+    assert z["k_fp4"] == 2 * 2 * 512 * 64 and z["vt_fp4"] == z["k_fp4"]
+    assert z["vt_sf"] == 2 * 2 * 4 * 1024 and z["k_mean"] == 2 * 2 * 128 * 4
+    assert z["amax"] == 3 * 2 * 8 * 4 and z["seq"] == 0
+    assert z["workspace"] >= sum(z[n] for n in ("q_fp4", "q_sf", "k_fp4", "k_sf", "vt_fp4", "vt_sf"))
+    zg = sage.problem_sizes(_dense_pr(sage, gscale="head"))
+    assert zg["scratch"] > z["scratch"]
+    # packed: bounded by both B * round128(max length) and total + 127 * B
+    torch = __import__("torch")
+    cu = torch.zeros(4, dtype=torch.int32)  # only its address is passed; nothing is read on the host
+    pr = _dense_pr(sage, B=3, Nq=1000, Nk=1000, cu_seqlens_q=cu, cu_seqlens_k=cu, total_q=1100,
+                   total_k=1100, q_stride=(0, 128, 8 * 128), k_stride=(0, 128, 2 * 128),
+                   v_stride=(0, 128, 2 * 128), o_stride=(0, 128, 8 * 128))
+    zp = sage.problem_sizes(pr)
+    rows = min(3 * 1024, (1100 + 127 * 3) // 128 * 128)
+    assert zp["q_fp4"] == 8 * rows * 64 and zp["seq"] == (2 * 4 + 4) * 4
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(Hkv=3), 1),                                  # Hq not a multiple of Hkv
+    (dict(D=96), 2),                                   # unsupported head dimension
+    (dict(q_stride=(8 * 300 * 128, 300 * 128, 100)), 1),  # token stride not 16-byte granular
+    (dict(gscale="none", sm_scale=float("inf")), 1),
+    (dict(Nq=-1), 1),
+])
+def test_general_problem_rejections(L, bad, status):
+    import microscaling_fp4_quantized_b200 as sage
+    with pytest.raises(sage.SageError) as e:
+        sage.problem_sizes(_dense_pr(sage, **bad))
+    assert e.value.status == status
+
+
+def test_packed_problem_needs_both_tables(L):
+    import microscaling_fp4_quantized_b200 as sage
+    torch = __import__("torch")
+    cu = torch.zeros(4, dtype=torch.int32)
+    with pytest.raises(sage.SageError) as e:
+        sage.problem_sizes(_dense_pr(sage, cu_seqlens_q=cu, total_q=10, total_k=10))
+    assert e.value.status == sage.SAGE_ERR_INVALID_ARG
