@@ -203,6 +203,71 @@ def run_reference(args, wl):
     return 0
 
 
+def run_sweep(args):
+    """Every named configuration once (tiny, medium, causal LLM, long, the 16-point sweep):
+    whole-forward and attention-only TOPS (CUDA events, median of 10 after 3 warm-ups),
+    parity against the oracle on sampled rows of the first and last head, and the
+    oracle's own rate on a bounded sample. One JSON line per configuration."""
+    import numpy as np
+    import oracle
+    import microscaling_fp4_quantized_b200 as sage
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks, basis = _peaks()
+    fp4_peak = FP4_PER_BF16 * peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    for wl in [workloads.TINY, workloads.MEDIUM, workloads.LLM_CAUSAL, workloads.LONG] + workloads.SWEEP:
+        q, k, v = workloads.make_inputs(wl)
+        qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+        out = torch.empty_like(qd)
+        plan = sage.Plan(wl.B, wl.H, wl.N, wl.D, wl.dtype, dev)
+        for _ in range(3):
+            plan.quantize(qd, kd, vd)
+            plan.attention(out, causal=wl.causal, sm_scale=wl.sm_scale)
+        torch.cuda.synchronize()
+        whole, attn = [], []
+        for _ in range(10):
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            e[0].record(stream)
+            plan.quantize(qd, kd, vd)
+            e[1].record(stream)
+            plan.attention(out, causal=wl.causal, sm_scale=wl.sm_scale)
+            e[2].record(stream)
+            whole.append(e)
+        torch.cuda.synchronize()
+        ms = statistics.median(a.elapsed_time(c) for a, _, c in whole)
+        ms_attn = statistics.median(b.elapsed_time(c) for _, b, c in whole)
+        err = sage.device_error()
+        BH = wl.B * wl.H
+        heads = sorted({0, BH - 1})
+        kmean = plan.k_mean[: BH * wl.D].reshape(BH, wl.D).cpu().numpy()
+        f = lambda t: t.float().reshape(BH, wl.N, wl.D)[heads].numpy()  # noqa: E731
+        qh, kh, vh = f(q), f(k), f(v)
+        rng = np.random.default_rng(wl.seed)
+        nr = wl.N if wl.N <= 256 else 32
+        rr = np.unique(np.concatenate([[0, wl.N - 1], rng.choice(wl.N, nr, replace=False)]))
+        rows = np.array([(i, r) for i in range(len(heads)) for r in rr], np.int64)
+        em, _ = oracle.attention(qh, kh, vh, wl.causal, wl.sm_scale, Bk=128, rows=rows,
+                                 kmean_in=kmean[heads])
+        ex = oracle.attn_exact(qh, kh, vh, wl.causal, wl.sm_scale, rows=rows)
+        og = out.float().reshape(BH, wl.N, wl.D)[heads].cpu().numpy()
+        got = og[rows[:, 0], rows[:, 1]]
+        m_em, m_ex = oracle.metrics(got, em), oracle.metrics(got, ex)
+        cpu_val, _, sample, cores = cpu_oracle_rate(wl, args.cpu_budget_s)
+        print(json.dumps({
+            "workload": wl.name, "ops": wl.ops, "tops": wl.ops / (ms * 1e-3) / 1e12, "ms": ms,
+            "attn_tops": wl.ops / (ms_attn * 1e-3) / 1e12, "attn_ms": ms_attn,
+            "pct_of_fp4_peak": 100.0 * wl.ops / (ms * 1e-3) / 1e12 / fp4_peak,
+            "peak_basis": f"{basis} bf16 sustained x {FP4_PER_BF16:g}",
+            "vs_emulated": {"cos": m_em["cos"], "max_abs_over_max_v": m_em["max_abs"] / float(np.abs(vh).max())},
+            "vs_exact": {"cos": m_ex["cos"], "rel_l1": m_ex["rel_l1"], "rmse": m_ex["rmse"]},
+            "sampled_rows": int(len(rows)), "device_error_word": err,
+            "cpu_oracle": {"value": cpu_val, "unit": UNIT, "cores": cores, "sample": sample}}), flush=True)
+        del qd, kd, vd, out, plan
+        torch.cuda.empty_cache()
+    return 0
+
+
 # Kernels per step: K statistics, K mean, quantization, attention.
 LAUNCHES_PER_STEP = 4
 
@@ -263,7 +328,12 @@ def main():
     ap.add_argument("--variants", action="store_true",
                     help="also time the general-problem paths (second-level scales, packed "
                          "grouped-query batch) and report them under 'variants'")
+    ap.add_argument("--sweep", action="store_true",
+                    help="measure every named configuration (one JSON line each) instead of "
+                         "the single bench line")
     args = ap.parse_args()
+    if args.sweep:
+        return run_sweep(args)
     wl = workloads.by_name(args.workload)
     if args.impl == "reference":
         return run_reference(args, wl)
