@@ -53,15 +53,38 @@ __device__ __forceinline__ uint4 ld_nc_16(const void* p) {
   return r;
 }
 
+// x / d rounded to nearest even, from r = RN(1/d): the FMA-corrected quotient of
+// Markstein ("IA-64 and Elementary Functions: Speed and Precision", 2000, ch. 8):
+// q = RN(x r), e = x - q d (exact with an FMA), result RN(q + e r). It is not correctly
+// rounded for every divisor, so it is used only where it was checked exhaustively on the
+// CPU against IEEE binary32 division: d = any positive E4M3 value with |x/d| in
+// [2^-4, 2^4) (E2M1 codes outside that range do not depend on the last bit of the
+// quotient), and d = 6 for every positive binary32 x with a normal quotient (a subnormal
+// a/6 gives scale byte 0 either way). The sign is copied from x so that -0 / d = -0.
+__device__ __forceinline__ float div_fma(float x, float d, float r) {
+  const float q = __fmul_rn(x, r);
+  const float e = __fmaf_rn(-q, d, x);
+  return copysignf(__fmaf_rn(e, r, q), x);
+}
+
+// RN(1/6) in binary32.
+constexpr float kRecip6 = 0.16666667163372039794921875f;
+
+// E4M3 scale byte of a block with maximum magnitude a: E4M3(RN(a / 6)).
+__device__ __forceinline__ uint32_t block_scale_byte(float a) {
+  return f32_to_e4m3(div_fma(a, 6.0f, kRecip6));
+}
+
 // Codes of 8 values against a decoded scale s (s == 0 -> zero codes); element 0 lands
-// in the low nibble of the low byte.
+// in the low nibble of the low byte. Each code is E2M1(RN(x / s)).
 __device__ __forceinline__ uint32_t encode8(const float (&x)[8], float s) {
   if (s == 0.0f) return 0u;
+  const float r = __frcp_rn(s);
   uint32_t w = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float a = __fdiv_rn(x[2 * i], s);
-    const float b = __fdiv_rn(x[2 * i + 1], s);
+    const float a = div_fma(x[2 * i], s, r);
+    const float b = div_fma(x[2 * i + 1], s, r);
     w |= f32x2_to_e2m1(a, b) << (8 * i);
   }
   return w;
@@ -190,6 +213,7 @@ __global__ void __launch_bounds__(kThreads) stats_kernel(QuantParams p) {
       mx[e] = -INFINITY;
       mn[e] = INFINITY;
     }
+#pragma unroll 4
     for (int n = n0 + rg; n < n1; n += RG) {
       float x[8];
       unpack8(ld_nc_16(row_ptr(p.k, p.sk, b, h, static_cast<int64_t>(si.tok_k) + n) + c * 16), p.dtype, x);
@@ -329,29 +353,39 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
     const void* src = job == 0 ? p.q : p.k;
     const Strides& st = job == 0 ? p.sq : p.sk;
     uint8_t* dst = (job == 0 ? p.q_fp4 : p.k_fp4) + row0 * (D / 2);
-#pragma unroll 2
-    for (int gi = t; gi < 128 * CPR; gi += kThreads) {
-      const int rl = gi / CPR, c = gi % CPR;
+    // Every thread owns one 8-channel chunk c of rows rl0, rl0 + kRowStep, ...: all of its
+    // 16-byte loads are issued before any of them is used.
+    constexpr int kRowStep = kThreads / CPR, kIter = 128 / kRowStep;
+    const int c = t % CPR, rl0 = t / CPR;
+    float m8[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m8[e] = mu[c * 8 + e];
+    uint4 raw[kIter];
+#pragma unroll
+    for (int it = 0; it < kIter; ++it) {
+      const int rl = rl0 + it * kRowStep;
+      raw[it] = rl < rows ? ld_nc_16(row_ptr(src, st, b, h, tok0 + rl) + c * 16) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int it = 0; it < kIter; ++it) {
+      const int rl = rl0 + it * kRowStep;
       float x[8];
+      unpack8(raw[it], p.dtype, x);
       if (rl < rows) {
-        unpack8(ld_nc_16(row_ptr(src, st, b, h, tok0 + rl) + c * 16), p.dtype, x);
         if (smooth) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], mu[c * 8 + e]);
+          for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], m8[e]);
         }
         if (gs) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) x[e] = __fdiv_rn(x[e], g);
         }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = 0.0f;
       }
       float a = 0.0f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(x[e]));
       a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));  // partner holds the other 8 of the block
-      const uint32_t sb = f32_to_e4m3(__fdiv_rn(a, 6.0f));
+      const uint32_t sb = block_scale_byte(a);
       const float s = e4m3_to_f32(sb);
       const uint32_t w = encode8(x, s);
       *reinterpret_cast<uint32_t*>(dst + static_cast<size_t>(rl) * (D / 2) + c * 4) = w;
@@ -372,11 +406,18 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
   uint8_t* cbuf = smem + 128 * kVRowBytes;              // D x kCodeRow
   uint8_t* sfbuf = cbuf + D * kCodeRow;                 // 1024
   for (int i = t; i < 1024 / 16; i += kThreads) reinterpret_cast<uint4*>(sfbuf)[i] = make_uint4(0, 0, 0, 0);
-  for (int gi = t; gi < 128 * CPR; gi += kThreads) {
-    const int rl = gi / CPR, c = gi % CPR;
-    uint4 raw = make_uint4(0, 0, 0, 0);
-    if (rl < rows) raw = ld_nc_16(row_ptr(p.v, p.sv, b, h, tok0 + rl) + c * 16);
-    *reinterpret_cast<uint4*>(vtile + rl * kVRowBytes + c * 16) = raw;
+  {
+    constexpr int kRowStep = kThreads / CPR, kIter = 128 / kRowStep;
+    const int c = t % CPR, rl0 = t / CPR;
+    uint4 raw[kIter];
+#pragma unroll
+    for (int it = 0; it < kIter; ++it) {
+      const int rl = rl0 + it * kRowStep;
+      raw[it] = rl < rows ? ld_nc_16(row_ptr(p.v, p.sv, b, h, tok0 + rl) + c * 16) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int it = 0; it < kIter; ++it)
+      *reinterpret_cast<uint4*>(vtile + (rl0 + it * kRowStep) * kVRowBytes + c * 16) = raw[it];
   }
   __syncthreads();
   for (int item = t; item < D * 8; item += kThreads) {
@@ -392,7 +433,7 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
     float a = 0.0f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(x[i]));
-    const uint32_t sb = f32_to_e4m3(__fdiv_rn(a, 6.0f));
+    const uint32_t sb = block_scale_byte(a);
     const float s = e4m3_to_f32(sb);
     float lo[8], hi[8];
 #pragma unroll

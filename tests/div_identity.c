@@ -1,0 +1,55 @@
+/* Checks the division identity the quantization kernel relies on (Markstein's
+ * FMA-corrected quotient, "IA-64 and Elementary Functions", ch. 8): with r = RN(1/d),
+ * q = RN(x r), e = x - q d (one FMA), RN(q + e r) with the sign of x equals the IEEE
+ * binary32 quotient x / d
+ *   - for every positive finite E4M3 divisor and every |x / d| in [2^-4, 2^4), visiting
+ *     every `stride`-th binary32 x (stride 1 = exhaustive), both signs, and x = -0;
+ *   - for d = 6 and every `stride`-th positive binary32 x whose quotient is normal.
+ * Prints the number of mismatches of each part; exit status 0 when both are 0. */
+#include <math.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+static float f_of(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+static uint32_t u_of(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+
+static double e4m3_value(int b) {
+  const int e = (b >> 3) & 15, m = b & 7;
+  return e == 0 ? ldexp(m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+}
+
+static float div_fma(float x, float d, float r) {
+  const float q = x * r;
+  const float e = fmaf(-q, d, x);
+  return copysignf(fmaf(e, r, q), x);
+}
+
+int main(int argc, char** argv) {
+  const uint32_t stride = argc > 1 ? (uint32_t)strtoul(argv[1], NULL, 10) : 1u;
+  long bad = 0, n = 0;
+  for (int b = 1; b <= 0x7E; ++b) {
+    const float d = (float)e4m3_value(b), r = 1.0f / d;
+    const uint32_t lo = u_of(d * 0.0625f), hi = u_of(d * 16.0f);
+    for (uint32_t u = lo; u < hi; u += stride) {
+      for (int sg = 0; sg < 2; ++sg) {
+        const float x = sg ? -f_of(u) : f_of(u);
+        if (u_of(div_fma(x, d, r)) != u_of(x / d)) ++bad;
+        ++n;
+      }
+    }
+    if (u_of(div_fma(-0.0f, d, r)) != u_of(-0.0f / d)) ++bad;
+    if (u_of(div_fma(0.0f, d, r)) != u_of(0.0f / d)) ++bad;
+    n += 2;
+  }
+  long bad6 = 0, n6 = 0;
+  const float r6 = 1.0f / 6.0f;
+  for (uint32_t u = 0x01000000u; u < 0x7F800000u; u += stride) {  /* a / 6 normal */
+    const float a = f_of(u);
+    if (u_of(div_fma(a, 6.0f, r6)) != u_of(a / 6.0f)) ++bad6;
+    ++n6;
+  }
+  printf("e4m3 divisors: %ld checks, %ld mismatches; d = 6: %ld checks, %ld mismatches\n", n, bad, n6, bad6);
+  return (bad == 0 && bad6 == 0) ? 0 : 1;
+}
