@@ -268,6 +268,75 @@ def run_sweep(args):
     return 0
 
 
+def time_e2e(sage, wl, q, k, v, dev, stream, steps, dist, world):
+    """End to end through the public API: every step copies its inputs from pinned host
+    memory, runs sage.attn, and copies the output back to pinned host memory.
+    Pipelined (the headline): a copy-in stream, the compute stream and a copy-out stream
+    with two device buffer sets, so step i+1's inputs and step i-1's output move while
+    step i computes -- a serving loop's schedule. Serial (reported beside it): the three
+    stages of each step back to back on one stream."""
+    hin = [(q.pin_memory(), k.pin_memory(), v.pin_memory()) for _ in range(2)]
+    hout = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(2)]
+    din = [tuple(torch.empty(q.shape, dtype=q.dtype, device=dev) for _ in range(3)) for _ in range(2)]
+    dout = [torch.empty(q.shape, dtype=q.dtype, device=dev) for _ in range(2)]
+    ws = torch.empty(max(sage.workspace_bytes(wl.B, wl.H, wl.N, wl.D), 256), dtype=torch.uint8, device=dev)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def pipelined(n):
+        ev_in = [torch.cuda.Event() for _ in range(n)]
+        ev_c = [torch.cuda.Event() for _ in range(n)]
+        ev_out = [torch.cuda.Event() for _ in range(n)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        s_in.wait_event(t0)
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_c[i - 2])          # buffer set b free again
+                for d, h in zip(din[b], hin[b]):
+                    d.copy_(h, non_blocking=True)
+                ev_in[i].record(s_in)
+            stream.wait_event(ev_in[i])
+            if i >= 2:
+                stream.wait_event(ev_out[i - 2])           # output buffer b read back
+            sage.attn(*din[b], causal=wl.causal, sm_scale=wl.sm_scale, out=dout[b], workspace=ws)
+            ev_c[i].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_c[i])
+                hout[b].copy_(dout[b], non_blocking=True)
+                ev_out[i].record(s_out)
+        stream.wait_event(ev_out[n - 1])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        return t0.elapsed_time(t1) / n
+
+    def serial(n):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(n):
+            a, b, c = (h.to(dev, non_blocking=True) for h in hin[0])
+            o = sage.attn(a, b, c, causal=wl.causal, sm_scale=wl.sm_scale)
+            hout[0].copy_(o, non_blocking=True)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        return t0.elapsed_time(t1) / n
+
+    pipelined(3)
+    serial(2)
+    if dist is not None:
+        dist.barrier()
+    ms_p = max_over_ranks(pipelined(steps), dist, dev)
+    ms_s = max_over_ranks(serial(steps), dist, dev)
+    if sage.device_error() != 0:
+        raise RuntimeError("device error word set in the end-to-end run")
+    nbytes = q.numel() * q.element_size()
+    return {"value": job_value(wl.ops, world, ms_p), "unit": UNIT, "ms_per_step": ms_p,
+            "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
+            "schedule": "pipelined: copy-in / compute / copy-out streams, two buffer sets",
+            "serial": {"value": job_value(wl.ops, world, ms_s), "ms_per_step": ms_s}}
+
+
 # Kernels per step: K statistics, K mean, quantization, attention.
 LAUNCHES_PER_STEP = 4
 
@@ -402,32 +471,7 @@ def main():
     # --- end to end through the public API: pinned host inputs -> result on the host ---
     e2e = None
     if not args.no_e2e:
-        qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
-        oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
-        e2e_steps = max(3, min(args.steps, 10))
-
-        def e2e_step():
-            a = qh.to(dev, non_blocking=True)
-            b = kh.to(dev, non_blocking=True)
-            c = vh.to(dev, non_blocking=True)
-            o = sage.attn(a, b, c, causal=wl.causal, sm_scale=wl.sm_scale)
-            oh.copy_(o, non_blocking=True)
-
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dist, dev)
-        nbytes = q.numel() * q.element_size()
-        e2e = {"value": job_value(wl.ops, world, e_ms), "unit": UNIT, "ms_per_step": e_ms,
-               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes}
+        e2e = time_e2e(sage, wl, q, k, v, dev, stream, max(3, args.steps), dist, world)
 
     variants = None
     if args.variants:
