@@ -62,8 +62,9 @@ def _L():
             "so_second_level_scale": [vp, c_long, vp],
             "so_quantize_rows": [vp, c_long, c_long, c_long, vp, vp, vp, vp],
             "so_quantize_vt": [vp, c_long, c_long, c_long, vp, vp, vp],
-            "so_attn_emulated": [vp, vp, vp, vp, vp, vp, vp, vp, vp, c_long, c_long, c_long,
+            "so_attn_emulated": [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, c_long, c_long, c_long,
                                  c_long, c_long, c_long, c_int, c_double, c_long, vp, c_long, vp],
+            "so_qk_bias": [vp, vp, vp, c_long, c_long, c_long, c_long, c_long, vp],
             "so_attn_exact": [vp, vp, vp, c_long, c_long, c_long, c_long, c_long, c_long, c_int,
                               c_double, vp, c_long, vp],
             "so_attn_online": [vp, vp, vp, c_long, c_long, c_long, c_int, c_double, c_long,
@@ -198,8 +199,20 @@ def quantize_vt(v, gscale=None):
 GSCALE_MODES = ("none", "tensor", "head")
 
 
+def qk_bias(mu_q, k, mu_k, heads) -> np.ndarray:
+    """The Q-smoothing bias [B*Hq, Nk] (binary64): mu_q . fp32(k - mu_k) per key."""
+    k = _f32(k)
+    B, Hq, Hkv = heads
+    BHkv, Nk, D = k.shape
+    mq = _f32(mu_q).reshape(B * Hq, D)
+    mk = None if mu_k is None else _f32(mu_k).reshape(BHkv, D)
+    out = np.empty((B * Hq, Nk), np.float64)
+    _L().so_qk_bias(_p(mq), _p(k), _p(mk) if mk is not None else None, B, Hq, Hkv, Nk, D, _p(out))
+    return out
+
+
 def quantize_qkv(q, k, v, smooth_k: bool = True, kmean_in=None, gscale: str = "none",
-                 amax_in=None, heads=None) -> dict:
+                 amax_in=None, heads=None, smooth_q: bool = False, qmean_in=None) -> dict:
     """Quantize one problem of equal-length sequences.
 
     q [B*Hq, Nq, D], k and v [B*Hkv, Nk, D] (float32 values of the bf16/fp16 inputs);
@@ -207,7 +220,9 @@ def quantize_qkv(q, k, v, smooth_k: bool = True, kmean_in=None, gscale: str = "n
     per-head token mean (kmean_in [B*Hkv, D] supplies it instead). gscale: "none", or a
     second-level scale per tensor ("tensor") or per head ("head") from the amax of Q,
     of the smoothed K and of V; amax_in = {"q": [B*Hq], "k": [B*Hkv], "v": [B*Hkv]}
-    supplies those maxima (already reduced for "tensor" mode).
+    supplies those maxima (already reduced for "tensor" mode). smooth_q: Q is quantized
+    as q - mu_q (mu_q its per-head token mean, qmean_in [B*Hq, D] supplies it) and the
+    emulation adds back qk_bias = mu_q . (k - mu_k) per key.
     """
     q, k, v = _f32(q), _f32(k), _f32(v)
     BHq, Nq, D = q.shape
@@ -219,18 +234,23 @@ def quantize_qkv(q, k, v, smooth_k: bool = True, kmean_in=None, gscale: str = "n
     km = np.zeros((BHkv, D), np.float32)
     if smooth_k:
         km = _f32(kmean_in).reshape(BHkv, D) if kmean_in is not None else kmean(k)
-    r = {"B": B, "Hq": Hq, "Hkv": Hkv, "Nq": Nq, "Nk": Nk, "D": D, "k_mean": km,
-         "gq": None, "gk": None, "gv": None, "amax": None}
+    qm = None
+    if smooth_q:
+        qm = _f32(qmean_in).reshape(BHq, D) if qmean_in is not None else kmean(q)
+    r = {"B": B, "Hq": Hq, "Hkv": Hkv, "Nq": Nq, "Nk": Nk, "D": D, "k_mean": km, "q_mean": qm,
+         "gq": None, "gk": None, "gv": None, "amax": None, "qk_bias": None}
+    if smooth_q:
+        r["qk_bias"] = qk_bias(qm, k, km if smooth_k else None, (B, Hq, Hkv))
     if gscale != "none":
         if amax_in is not None:
             am = {n: _f32(amax_in[n]).ravel() for n in ("q", "k", "v")}
         else:
-            am = {"q": group_amax(q), "k": group_amax(k, km if smooth_k else None), "v": group_amax(v)}
+            am = {"q": group_amax(q, qm), "k": group_amax(k, km if smooth_k else None), "v": group_amax(v)}
             if gscale == "tensor":
                 am = {n: np.full(a.shape, a.max(initial=0.0), np.float32) for n, a in am.items()}
         r["amax"] = am
         r["gq"], r["gk"], r["gv"] = (second_level_scale(am[n]) for n in ("q", "k", "v"))
-    r["q_codes"], r["q_sf"] = quantize_rows(q, None, r["gq"])
+    r["q_codes"], r["q_sf"] = quantize_rows(q, qm, r["gq"])
     r["k_codes"], r["k_sf"] = quantize_rows(k, km if smooth_k else None, r["gk"])
     r["vt_codes"], r["vt_sf"] = quantize_vt(v, r["gv"])
     return r
@@ -253,7 +273,10 @@ def attn_emulated(qz: dict, causal: bool, sm_scale: float, Bk: int = 128, rows=N
     out = np.empty((r.shape[0], D), np.float64)
     arrs = [np.ascontiguousarray(qz[n]) for n in ("q_codes", "q_sf", "k_codes", "k_sf", "vt_codes", "vt_sf")]
     gs = [None if qz[n] is None else _f32(qz[n]) for n in ("gq", "gk", "gv")]
+    bias = qz.get("qk_bias")
+    bias = None if bias is None else np.ascontiguousarray(bias, dtype=np.float64)
     _L().so_attn_emulated(*[_p(a) for a in arrs], *[_p(g) if g is not None else None for g in gs],
+                          _p(bias) if bias is not None else None,
                           B, Hq, Hkv, Nq, Nk, D, int(bool(causal)), float(sm_scale), int(Bk),
                           _p(r), r.shape[0], _p(out))
     return out.reshape(B * Hq, Nq, D) if rows is None else out
@@ -286,17 +309,19 @@ def attn_online(q, k, v, causal: bool, sm_scale: float, Bk: int = 128, rows=None
 
 def attention(q, k, v, causal: bool, sm_scale: float, Bk: int = 128, rows=None,
               smooth_k: bool = True, kmean_in=None, gscale: str = "none", heads=None,
-              amax_in=None):
+              amax_in=None, smooth_q: bool = False, qmean_in=None):
     """Full emulated pipeline: K mean, block quantization, emulated FP4 attention."""
     qz = quantize_qkv(q, k, v, smooth_k=smooth_k, kmean_in=kmean_in, gscale=gscale,
-                      amax_in=amax_in, heads=heads)
+                      amax_in=amax_in, heads=heads, smooth_q=smooth_q, qmean_in=qmean_in)
     return attn_emulated(qz, causal, sm_scale, Bk=Bk, rows=rows), qz
 
 
-def varlen_amax(q, k, v, cu_q, cu_k, smooth_k: bool = True, kmeans=None) -> dict:
+def varlen_amax(q, k, v, cu_q, cu_k, smooth_k: bool = True, kmeans=None, smooth_q: bool = False,
+                qmeans=None) -> dict:
     """Per-tensor maxima of packed sequences (q [Tq, Hq, D], k, v [Tk, Hkv, D]) for the
-    "tensor" second-level scale: max over every sequence and head, K smoothed by the
-    mean of its own sequence (kmeans[b] [Hkv, D] supplies those)."""
+    "tensor" second-level scale: max over every sequence and head, K (and Q with
+    smooth_q) smoothed by the mean of its own sequence (kmeans[b] [Hkv, D] and qmeans[b]
+    [Hq, D] supply those)."""
     a = {"q": 0.0, "k": 0.0, "v": 0.0}
     for b in range(len(cu_q) - 1):
         qs = _f32(q[cu_q[b]:cu_q[b + 1]]).transpose(1, 0, 2)
@@ -306,7 +331,10 @@ def varlen_amax(q, k, v, cu_q, cu_k, smooth_k: bool = True, kmeans=None) -> dict
         if smooth_k and ks.shape[1] > 0:
             km = kmeans[b] if kmeans is not None else kmean(ks)
         if qs.shape[1] > 0:
-            a["q"] = max(a["q"], float(group_amax(qs).max()))
+            qm = None
+            if smooth_q:
+                qm = qmeans[b] if qmeans is not None else kmean(qs)
+            a["q"] = max(a["q"], float(group_amax(qs, qm).max()))
         if ks.shape[1] > 0:
             a["k"] = max(a["k"], float(group_amax(ks, km).max()))
             a["v"] = max(a["v"], float(group_amax(vs).max()))
@@ -314,7 +342,8 @@ def varlen_amax(q, k, v, cu_q, cu_k, smooth_k: bool = True, kmeans=None) -> dict
 
 
 def attention_varlen(q, k, v, cu_q, cu_k, causal: bool, sm_scale: float, Bk: int = 128,
-                     smooth_k: bool = True, gscale: str = "none", kmeans=None, rows=None):
+                     smooth_k: bool = True, gscale: str = "none", kmeans=None, rows=None,
+                     smooth_q: bool = False, qmeans=None):
     """Packed variable-length sequences, each an independent problem.
 
     q [Tq, Hq, D], k and v [Tk, Hkv, D]; sequence b holds query tokens cu_q[b]..cu_q[b+1]
@@ -329,7 +358,7 @@ def attention_varlen(q, k, v, cu_q, cu_k, causal: bool, sm_scale: float, Bk: int
     nseq = len(cu_q) - 1
     am = None
     if gscale == "tensor":
-        t = varlen_amax(q, k, v, cu_q, cu_k, smooth_k, kmeans)
+        t = varlen_amax(q, k, v, cu_q, cu_k, smooth_k, kmeans, smooth_q, qmeans)
     want = np.asarray(rows, np.int64).reshape(-1, 2) if rows is not None else None
     full = np.zeros((Tq, Hq, D), np.float64)
     qzs = []
@@ -353,7 +382,8 @@ def attention_varlen(q, k, v, cu_q, cu_k, causal: bool, sm_scale: float, Bk: int
             sel = np.stack([want[m, 1], want[m, 0] - cu_q[b]], 1)
         o, qz = attention(qs, ks, vs, causal, sm_scale, Bk=Bk, rows=sel, smooth_k=smooth_k,
                           kmean_in=None if kmeans is None else kmeans[b], gscale=gscale,
-                          heads=(1, Hq, Hkv), amax_in=am)
+                          heads=(1, Hq, Hkv), amax_in=am, smooth_q=smooth_q,
+                          qmean_in=None if qmeans is None else qmeans[b])
         qzs.append(qz)
         if sel is None:
             full[cu_q[b]:cu_q[b + 1]] = o.transpose(1, 0, 2)

@@ -263,14 +263,42 @@ void so_quantize_vt(const float* v, long G, long N, long D, const float* gscale,
   }
 }
 
+// ------------------------------------------------------------ Q smoothing ----
+// Smoothing Q (named in the SageAttention2 abstract on the author page, the counterpart
+// of smoothing K): each query row is quantized as q' = fp32(q - mu_q), mu_q the channel
+// mean of the (sequence, query head) -- computed by so_kmean on Q -- and the part that
+// was taken out returns as a per-key bias of the scores,
+//   bias[bhq, j] = sum_d mu_q[bhq, d] * k'[kv(bhq), j, d]      (binary64),
+// with k' = fp32(k - mu_k) the smoothed, unquantized keys (k itself when mu_k is NULL),
+// so that q . k' = q' . k' + bias exactly. kv(bhq) follows the grouped-head map of
+// so_attn_emulated. mu_q [B*Hq, D]; k [B*Hkv, Nk, D]; mu_k [B*Hkv, D]; bias [B*Hq, Nk].
+void so_qk_bias(const float* mu_q, const float* k, const float* mu_k, long B, long Hq, long Hkv,
+                long Nk, long D, double* bias) {
+  const long group = Hq / Hkv;
+#pragma omp parallel for schedule(static)
+  for (long bhq = 0; bhq < B * Hq; ++bhq) {
+    const long kv = (bhq / Hq) * Hkv + (bhq % Hq) / group;
+    for (long j = 0; j < Nk; ++j) {
+      double acc = 0.0;
+      for (long d = 0; d < D; ++d) {
+        float kk = k[(kv * Nk + j) * D + d];
+        if (mu_k) kk = kk - mu_k[kv * D + d];
+        acc += static_cast<double>(mu_q[bhq * D + d]) * static_cast<double>(kk);
+      }
+      bias[bhq * Nk + j] = acc;
+    }
+  }
+}
+
 // ------------------------------------------------------ emulated attention ----
 // One or more sequences of equal lengths: B batches, Hq query heads, Hkv key/value heads
 // (query head h reads key/value head h / (Hq / Hkv)), Nq queries and Nk keys each.
 // Arrays: q codes/sf [B*Hq, Nq, ...]; k codes/sf [B*Hkv, Nk, ...]; vt [B*Hkv, D, ...];
-// gq [B*Hq], gk, gv [B*Hkv] second-level scales (NULL = 1).
+// gq [B*Hq], gk, gv [B*Hkv] second-level scales (NULL = 1); qk_bias [B*Hq, Nk] the Q
+// smoothing bias of so_qk_bias (NULL = none), added to the dot product before sm_scale.
 // For each requested row (bhq, i): dequantize exactly in binary64 (code * scale * g)
 // and walk key tiles of width Bk (the GPU kernel's key-tile width) from key 0:
-//   S_j   = sm_scale * sum_d q~_id k~_jd                      (binary64)
+//   S_j   = sm_scale * (sum_d q~_id k~_jd + qk_bias_j)         (binary64)
 //   m'    = max(m, max_j S_j)   (masked keys excluded)
 //   P~_j  = exp(S_j - m')                                      (masked keys -> 0)
 //   l     = l * exp(m - m') + sum_j P~_j                       (unquantized P~)
@@ -282,9 +310,9 @@ void so_quantize_vt(const float* v, long G, long N, long D, const float* gscale,
 // rows: n_rows pairs (bhq, i); out: [n_rows, D] binary64.
 void so_attn_emulated(const uint8_t* q_codes, const uint8_t* q_sf, const uint8_t* k_codes,
                       const uint8_t* k_sf, const uint8_t* vt_codes, const uint8_t* vt_sf,
-                      const float* gq, const float* gk, const float* gv, long B, long Hq,
-                      long Hkv, long Nq, long Nk, long D, int causal, double sm_scale, long Bk,
-                      const long* rows, long n_rows, double* out) {
+                      const float* gq, const float* gk, const float* gv, const double* qk_bias,
+                      long B, long Hq, long Hkv, long Nq, long Nk, long D, int causal,
+                      double sm_scale, long Bk, const long* rows, long n_rows, double* out) {
   (void)B;
   const long group = Hq / Hkv;
   const long Nkp = (Nk + 15) / 16 * 16;
@@ -339,6 +367,7 @@ void so_attn_emulated(const uint8_t* q_codes, const uint8_t* q_sf, const uint8_t
         for (long j = j0; j < j1; ++j) {
           double acc = 0.0;
           for (long d = 0; d < D; ++d) acc += qd[d] * kd[j * D + d];
+          if (qk_bias) acc += qk_bias[bhq * Nk + j];
           S[j - j0] = sm_scale * acc;
           tmax = std::max(tmax, S[j - j0]);
         }
