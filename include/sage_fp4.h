@@ -22,6 +22,10 @@
  *      page, "TetraJet-v2" abstract: double-block quantization for NVFP4), applied the
  *      way step 4 scales P~: g = amax / (448*6), the 16-element rule runs on x / g, and
  *      g is folded back into the scores (Q, K) and the output (V).
+ *   6. Optional (sage_fp4_problem_t.smooth_q): smoothing Q (SageAttention2 abstract on the
+ *      author page), read as the counterpart of step 1: Q' = Q - mean_over_tokens(Q) is
+ *      quantized, and the removed part returns as a per-key score bias mu_q . K' computed
+ *      from the unquantized smoothed keys (one FP32 add per score).
  *
  * Conventions for every entry point
  *   - Tensors are device pointers unless stated; the caller owns all memory. The
@@ -124,6 +128,8 @@ typedef struct {
   float sm_scale;               /* <= 0: 1/sqrt(D) */
   int smooth_k;                 /* subtract the per-(sequence, head) channel mean of K */
   sage_gscale_t gscale;
+  int smooth_q;                 /* subtract the per-(sequence, head) channel mean of Q before
+                                   quantizing it, and add mu_q . (k - mu_k) back to the scores */
 } sage_fp4_problem_t;
 
 /* The quantized tensors of a problem (layouts above); device pointers, 16-byte aligned. */
@@ -133,12 +139,21 @@ typedef struct {
   float* amax;                  /* required when gscale != SAGE_GSCALE_NONE */
   int32_t* seq;                 /* packed problems: the padded offsets of every sequence,
                                    [2, B+1] int32 plus a validity word; else unused */
+  float* q_mean;                /* smooth_q: [B*Hq, D] query means */
+  uint8_t* qk_bias;             /* smooth_q: 32 bytes per query head and padded key row (the
+                                   key rows' layout with Hq heads): b = mu_q . (k - mu_k)
+                                   divided by the Q and K second-level scales (1 without), as
+                                   bf16 terms hi, mid, lo (hi = bf16(b), mid = bf16(b - hi),
+                                   lo = bf16(b - hi - mid)) in elements 0-2 of 16, zeros
+                                   after; the 128 keys of a tile form a 4 KiB tensor-core
+                                   operand: key n, 8-element half c at byte
+                                   (n/8)*256 + c*128 + (n%8)*16 of the tile */
 } sage_fp4_quantized_t;
 
 /* Byte sizes for a problem (all 0 for an empty problem). For packed problems the
  * quantized sizes are upper bounds computed from B, Nq, Nk, total_q and total_k. */
 typedef struct {
-  size_t q_fp4, q_sf, k_fp4, k_sf, vt_fp4, vt_sf, k_mean, amax, seq;
+  size_t q_fp4, q_sf, k_fp4, k_sf, vt_fp4, vt_sf, k_mean, amax, seq, q_mean, qk_bias;
   size_t scratch;    /* scratch of sage_fp4_quantize */
   size_t workspace;  /* workspace of sage_fp4_attn: the above, each 256-byte aligned */
 } sage_fp4_problem_sizes_t;

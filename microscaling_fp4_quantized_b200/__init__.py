@@ -64,10 +64,11 @@ class _Problem(ctypes.Structure):
                 ("q_stride", ctypes.c_int64 * 3), ("k_stride", ctypes.c_int64 * 3),
                 ("v_stride", ctypes.c_int64 * 3), ("o_stride", ctypes.c_int64 * 3),
                 ("dtype", ctypes.c_int), ("causal", ctypes.c_int), ("sm_scale", ctypes.c_float),
-                ("smooth_k", ctypes.c_int), ("gscale", ctypes.c_int)]
+                ("smooth_k", ctypes.c_int), ("gscale", ctypes.c_int), ("smooth_q", ctypes.c_int)]
 
 
-_QZ_FIELDS = ("q_fp4", "q_sf", "k_fp4", "k_sf", "vt_fp4", "vt_sf", "k_mean", "amax", "seq")
+_QZ_FIELDS = ("q_fp4", "q_sf", "k_fp4", "k_sf", "vt_fp4", "vt_sf", "k_mean", "amax", "seq", "q_mean",
+              "qk_bias")
 
 
 class _Quantized(ctypes.Structure):
@@ -338,7 +339,7 @@ def make_problem(*, B: int, Hq: int, Hkv: int, D: int, Nq: int, Nk: int, dtype: 
                  sm_scale: Optional[float] = None, smooth_k: bool = True, gscale: str = "none",
                  cu_seqlens_q: Optional[torch.Tensor] = None,
                  cu_seqlens_k: Optional[torch.Tensor] = None, total_q: int = 0,
-                 total_k: int = 0) -> _Problem:
+                 total_k: int = 0, smooth_q: bool = False) -> _Problem:
     """The C problem descriptor (strides in elements of (sequence, head, token))."""
     if gscale not in GSCALE:
         raise ValueError(f"gscale must be one of {tuple(GSCALE)}")
@@ -357,6 +358,7 @@ def make_problem(*, B: int, Hq: int, Hkv: int, D: int, Nq: int, Nk: int, dtype: 
     pr.sm_scale = float(sm_scale or 0.0)
     pr.smooth_k = int(bool(smooth_k))
     pr.gscale = GSCALE[gscale]
+    pr.smooth_q = int(bool(smooth_q))
     return pr
 
 
@@ -379,6 +381,7 @@ def quantize(pr: _Problem, q, k, v) -> dict:
     buf["k_mean"] = buf["k_mean"].view(torch.float32)
     buf["amax"] = buf["amax"].view(torch.float32)
     buf["seq"] = buf["seq"].view(torch.int32)
+    buf["q_mean"] = buf["q_mean"].view(torch.float32)
     buf["problem"] = pr
     return buf
 
@@ -413,7 +416,7 @@ def _same_kind(q, k, v):
 
 def sageattn_problem(q, k, v, out, tensor_layout: str = "HND", is_causal: bool = False,
                      sm_scale: Optional[float] = None, smooth_k: bool = True,
-                     gscale: str = "none") -> _Problem:
+                     gscale: str = "none", smooth_q: bool = False) -> _Problem:
     """The problem descriptor :func:`sageattn` passes to the library."""
     _same_kind(q, k, v)
     if tensor_layout == "HND":
@@ -431,28 +434,29 @@ def sageattn_problem(q, k, v, out, tensor_layout: str = "HND", is_causal: bool =
     return make_problem(B=B, Hq=Hq, Hkv=Hkv, D=D, Nq=Nq, Nk=Nk, dtype=q.dtype,
                         q_stride=_strides3(q, dims), k_stride=_strides3(k, dims),
                         v_stride=_strides3(v, dims), o_stride=_strides3(out, dims), causal=is_causal,
-                        sm_scale=sm_scale, smooth_k=smooth_k, gscale=gscale)
+                        sm_scale=sm_scale, smooth_k=smooth_k, gscale=gscale, smooth_q=smooth_q)
 
 
 def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tensor_layout: str = "HND",
              is_causal: bool = False, sm_scale: Optional[float] = None, smooth_k: bool = True,
              gscale: str = "none", out: Optional[torch.Tensor] = None,
-             workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+             workspace: Optional[torch.Tensor] = None, smooth_q: bool = False) -> torch.Tensor:
     """FP4 attention on [B, H, N, D] ("HND") or [B, N, H, D] ("NHD") tensors with any
     strides (channels contiguous). k and v may have fewer heads than q (each shared by
     Hq / Hkv query heads) and a different length (the causal mask then aligns the last
     query with the last key). gscale adds a second-level FP32 scale per tensor ("tensor")
-    or per (batch, head) ("head")."""
+    or per (batch, head) ("head"); smooth_q subtracts each head's query mean before
+    quantization and adds its product with the keys back to the scores."""
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype, device=q.device)
-    pr = sageattn_problem(q, k, v, out, tensor_layout, is_causal, sm_scale, smooth_k, gscale)
+    pr = sageattn_problem(q, k, v, out, tensor_layout, is_causal, sm_scale, smooth_k, gscale, smooth_q)
     return _run(pr, q, k, v, out, workspace)
 
 
 def sageattn_varlen_problem(q, k, v, out, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
                             max_seqlen_k: int, is_causal: bool = False,
                             sm_scale: Optional[float] = None, smooth_k: bool = True,
-                            gscale: str = "none") -> _Problem:
+                            gscale: str = "none", smooth_q: bool = False) -> _Problem:
     """The problem descriptor :func:`sageattn_varlen` passes to the library."""
     _same_kind(q, k, v)
     if q.dim() != 3 or k.dim() != 3:
@@ -470,7 +474,8 @@ def sageattn_varlen_problem(q, k, v, out, cu_seqlens_q, cu_seqlens_k, max_seqlen
                       k_stride=_strides3(k, dims), v_stride=_strides3(v, dims),
                       o_stride=_strides3(out, dims), causal=is_causal, sm_scale=sm_scale,
                       smooth_k=smooth_k, gscale=gscale, cu_seqlens_q=cu_seqlens_q,
-                      cu_seqlens_k=cu_seqlens_k, total_q=total_q, total_k=total_k)
+                      cu_seqlens_k=cu_seqlens_k, total_q=total_q, total_k=total_k,
+                      smooth_q=smooth_q)
 
 
 def sageattn_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.Tensor,
@@ -478,7 +483,7 @@ def sageattn_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
                     is_causal: bool = False, sm_scale: Optional[float] = None,
                     smooth_k: bool = True, gscale: str = "none",
                     out: Optional[torch.Tensor] = None,
-                    workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+                    workspace: Optional[torch.Tensor] = None, smooth_q: bool = False) -> torch.Tensor:
     """FP4 attention on packed sequences: q [total_q, Hq, D], k and v [total_k, Hkv, D];
     sequence b holds tokens cu_seqlens_q[b] .. cu_seqlens_q[b+1] (int32 CUDA tensors of
     B+1 offsets; a bad table is reported by device_error(), never by a fault). Each
@@ -486,5 +491,5 @@ def sageattn_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype, device=q.device)
     pr = sageattn_varlen_problem(q, k, v, out, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
-                                 max_seqlen_k, is_causal, sm_scale, smooth_k, gscale)
+                                 max_seqlen_k, is_causal, sm_scale, smooth_k, gscale, smooth_q)
     return _run(pr, q, k, v, out, workspace)

@@ -56,8 +56,11 @@ constexpr uint32_t kColSfK = 392;   // + 8 * stage
 constexpr uint32_t kColSfV = 416;   // + 8 * stage
 constexpr uint32_t kColSfP = 440;   // + 8 * P buffer
 
-template <int D>
+template <int D, bool QB = false>
 struct Layout {
+  // QB: the Q-smoothing instance, which adds the score bias with one bf16 MMA per key tile.
+  static constexpr int kBiasBytes = QB ? 4096 : 0;   // per stage: 128 keys x 16 bf16, core-matrix layout
+  static constexpr int kOnesBytes = QB ? 4096 : 0;   // 128 rows x 16 bf16: ones in columns 0-2
   static constexpr int kQBytes = 128 * D / 2;
   static constexpr int kSfQKBytes = (D / 64) * 512;
   static constexpr int kKBytes = 128 * D / 2;
@@ -71,13 +74,15 @@ struct Layout {
   static constexpr int st_sfk = align1k(kKBytes);
   static constexpr int st_v = align1k(st_sfk + kSfQKBytes);
   static constexpr int st_sfv = align1k(st_v + kVBytes);
-  static constexpr int kStageBytes = align1k(st_sfv + kSfVBytes);
+  static constexpr int st_bias = align1k(st_sfv + kSfVBytes);
+  static constexpr int kStageBytes = align1k(st_bias + kBiasBytes);
   static constexpr int off_stage = align1k(off_sfq + kSfQKBytes);
   static constexpr int off_p = off_stage + kStages * kStageBytes;
   static constexpr int off_sfp = off_p + 2 * kPBytes;
   static constexpr int off_xch = off_sfp + 2 * kSfPBytes;  // [2 tiles][2 halves][128] floats
   static constexpr int off_lsum = off_xch + 2 * 2 * 128 * 4;  // [2 halves][128] floats
-  static constexpr int off_bar = off_lsum + 2 * 128 * 4;
+  static constexpr int off_ones = align1k(off_lsum + 2 * 128 * 4);
+  static constexpr int off_bar = off_ones + kOnesBytes;
   static constexpr int kNumBars = 32;
   static constexpr int off_misc = off_bar + kNumBars * 8;    // tmem base, abort flag
   static constexpr int kBytes = off_misc + 16;
@@ -172,11 +177,15 @@ __device__ __forceinline__ void store_out8(void* out, size_t idx, const float* v
 
 }  // namespace
 
-template <int D, bool CAUSAL, bool GENERAL>
+// MODE 0: square dense, one-level scales; 1: general; 2: general with the Q-smoothing
+// score bias.
+template <int D, bool CAUSAL, int MODE>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fp4_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
-  using L = Layout<D>;
+  constexpr bool GENERAL = MODE >= 1;
+  constexpr bool QBIAS = MODE == 2;
+  using L = Layout<D, QBIAS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -214,6 +223,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // those rows index the scale-factor tiles and the V^T tiles.
   const int qrow0 = p.Hq * si.prow_q + hq * nqt * 128 + qt * 128;
   const int ktile0 = (p.Hkv * si.prow_k + hk * nkt * 128) >> 7;
+  // Q-smoothing bias of (query head, key tile 0): 32 bytes (16 bf16) per padded key row.
+  const size_t bias_row0 = static_cast<size_t>(p.Hq) * si.prow_k + static_cast<size_t>(hq) * nkt * 128;
   Ctl ctl{misc + 1, p.err, p.timeout_ns};
 
   if (threadIdx.x == 0) {
@@ -246,6 +257,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tmem_alloc(sbase + L::off_misc, kTmemCols);
     tmem_relinquish();
   }
+  if (QBIAS && threadIdx.x < 128) {
+    // A operand of the bias MMA: every row (1, 1, 1, 0, ...) in bf16, so that
+    // S += A B^T adds the three bf16 terms of each key's bias to every query row.
+    // Core-matrix layout (no swizzle): row r, 16-byte half c at (r/8)*256 + c*128 + (r%8)*16.
+    const int r = threadIdx.x;
+    uint8_t* row = smem + L::off_ones + (r >> 3) * 256 + (r & 7) * 16;
+    *reinterpret_cast<uint4*>(row) = make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u);
+    *reinterpret_cast<uint4*>(row + 128) = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -264,10 +285,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int st = j % kStages;
         if (!wait_bar(bar(B_KVEMPTY + st), ((j / kStages) & 1) ^ 1, ctl)) break;
         const uint32_t sst = sbase + L::off_stage + st * L::kStageBytes;
-        mbar_arrive_expect_tx(bar(B_KFULL + st), L::kKBytes + L::kSfQKBytes);
+        mbar_arrive_expect_tx(bar(B_KFULL + st), L::kKBytes + L::kSfQKBytes + L::kBiasBytes);
         tma_load_2d(sst + L::st_k, &tm_k, 0, (ktile0 + j) * 128, bar(B_KFULL + st));
         bulk_load(sst + L::st_sfk, p.k_sf + static_cast<size_t>(ktile0 + j) * L::kSfQKBytes,
                   L::kSfQKBytes, bar(B_KFULL + st));
+        if (QBIAS)
+          bulk_load(sst + L::st_bias, p.qk_bias + (bias_row0 + static_cast<size_t>(j) * 128) * 32, L::kBiasBytes,
+                    bar(B_KFULL + st));
         mbar_arrive_expect_tx(bar(B_VFULL + st), L::kVBytes + L::kSfVBytes);
         tma_load_2d(sst + L::st_v, &tm_v, 0, (ktile0 + j) * D, bar(B_VFULL + st));
         bulk_load(sst + L::st_sfv, p.vt_sf + static_cast<size_t>(ktile0 + j) * L::kSfVBytes,
@@ -310,6 +334,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tc_mma_fp4(tmem + kColS0 + 128 * sb, qk_desc<D>(sbase + L::off_q + 32 * c),
                        qk_desc<D>(sst + L::st_k + 32 * c), idesc_s, tmem + kColSfQ + 4 * c,
                        tmem + kColSfK + 8 * st + 4 * c, c > 0 ? 1u : 0u);
+          if (QBIAS)  // S += ones * bias^T: the Q-smoothing bias of each key, on the tensor core
+            tc_mma_bf16(tmem + kColS0 + 128 * sb, make_sdesc(sbase + L::off_ones, 128, 256, kLayoutNone),
+                        make_sdesc(sst + L::st_bias, 128, 256, kLayoutNone), make_idesc_bf16(128), 1u);
           tc_commit(bar(B_SFULL + sb));
         }
         if (j >= 1) {
@@ -633,37 +660,43 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-template <int D>
+template <int D, bool QB>
 static int attn_smem_bytes() {
-  const int need = Layout<D>::kBytes + 1024;
+  const int need = Layout<D, QB>::kBytes + 1024;
   // At least 116 KiB so that two CTAs never share an SM (each holds all 512 TMEM columns).
   return need > 116 * 1024 ? need : 116 * 1024;
 }
 
-template <int D, bool CAUSAL, bool GENERAL>
+template <int D, bool CAUSAL, int MODE>
 static cudaError_t launch_attn_t(const TensorMaps& m, const AttnParams& p, int tiles_q, cudaStream_t stream) {
-  const int smem = attn_smem_bytes<D>();
-  cudaError_t e = cudaFuncSetAttribute(attn_fp4_fwd_kernel<D, CAUSAL, GENERAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int smem = attn_smem_bytes<D, MODE == 2>();
+  cudaError_t e = cudaFuncSetAttribute(attn_fp4_fwd_kernel<D, CAUSAL, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(tiles_q, p.Hq, p.B);
-  attn_fp4_fwd_kernel<D, CAUSAL, GENERAL><<<grid, kAttnThreads, smem, stream>>>(m.q, m.k, m.v, p);
+  attn_fp4_fwd_kernel<D, CAUSAL, MODE><<<grid, kAttnThreads, smem, stream>>>(m.q, m.k, m.v, p);
   return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_attn_d(const TensorMaps& m, const AttnParams& p, int tiles_q, int mode, cudaStream_t stream) {
+  if (p.causal) {
+    if (mode == 2) return launch_attn_t<D, true, 2>(m, p, tiles_q, stream);
+    if (mode == 1) return launch_attn_t<D, true, 1>(m, p, tiles_q, stream);
+    return launch_attn_t<D, true, 0>(m, p, tiles_q, stream);
+  }
+  if (mode == 2) return launch_attn_t<D, false, 2>(m, p, tiles_q, stream);
+  if (mode == 1) return launch_attn_t<D, false, 1>(m, p, tiles_q, stream);
+  return launch_attn_t<D, false, 0>(m, p, tiles_q, stream);
 }
 
 cudaError_t launch_attention(const TensorMaps& m, const AttnParams& p, int tiles_q, cudaStream_t stream) {
   if (p.B == 0 || p.Hq == 0 || tiles_q == 0) return cudaSuccess;
-  // The general instance serves packed sequences, Nq != Nk and second-level scales; a
-  // square dense problem with one-level scales gets the leaner loop (constant score
-  // scale, no mask offset, no empty-row guard).
+  // The general instance serves packed sequences, Nq != Nk and second-level scales, the
+  // third one adds the Q-smoothing bias; a square dense problem with one-level scales
+  // gets the leaner loop (constant score scale, no mask offset, no empty-row guard).
   const bool general = p.seq.cu_q != nullptr || p.seq.Nq != p.seq.Nk || p.amax != nullptr;
-  if (p.D == 64) {
-    if (general)
-      return p.causal ? launch_attn_t<64, true, true>(m, p, tiles_q, stream) : launch_attn_t<64, false, true>(m, p, tiles_q, stream);
-    return p.causal ? launch_attn_t<64, true, false>(m, p, tiles_q, stream) : launch_attn_t<64, false, false>(m, p, tiles_q, stream);
-  }
-  if (general)
-    return p.causal ? launch_attn_t<128, true, true>(m, p, tiles_q, stream) : launch_attn_t<128, false, true>(m, p, tiles_q, stream);
-  return p.causal ? launch_attn_t<128, true, false>(m, p, tiles_q, stream) : launch_attn_t<128, false, false>(m, p, tiles_q, stream);
+  const int mode = p.qk_bias != nullptr ? 2 : (general ? 1 : 0);
+  return p.D == 64 ? launch_attn_d<64>(m, p, tiles_q, mode, stream) : launch_attn_d<128>(m, p, tiles_q, mode, stream);
 }
 
 template <int D>

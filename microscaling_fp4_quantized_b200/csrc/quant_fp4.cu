@@ -184,10 +184,65 @@ __global__ void __launch_bounds__(1024) seq_plan_kernel(QuantParams p) {
   if (t == 0) *p.bad_out = 0u;
 }
 
+// Channel statistics of one 512-token chunk of one (sequence, head) of a [.., D] input:
+// binary64 sums into sum[.., D]; with extremes also float maxima / minima per channel.
+template <int D>
+__device__ __forceinline__ void chunk_channel_stats(const void* src, const Strides& st, int dtype, int b, int h,
+                                                    int64_t tok0, int n0, int n1, bool extremes,
+                                                    double* sum, float* cmax, float* cmin,
+                                                    double (*red)[D], float (*redmx)[D], float (*redmn)[D]) {
+  constexpr int CPR = D / 8;
+  constexpr int RG = kThreads / CPR;
+  const int t = threadIdx.x, c = t % CPR, rg = t / CPR;
+  double acc[8];
+  float mx[8], mn[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    acc[e] = 0.0;
+    mx[e] = -INFINITY;
+    mn[e] = INFINITY;
+  }
+#pragma unroll 4
+  for (int n = n0 + rg; n < n1; n += RG) {
+    float x[8];
+    unpack8(ld_nc_16(row_ptr(src, st, b, h, tok0 + n) + c * 16), dtype, x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      acc[e] += static_cast<double>(x[e]);
+      mx[e] = fmaxf(mx[e], x[e]);
+      mn[e] = fminf(mn[e], x[e]);
+    }
+  }
+  __syncthreads();  // the reduction buffers may still be read by a previous call
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    red[rg][c * 8 + e] = acc[e];
+    redmx[rg][c * 8 + e] = mx[e];
+    redmn[rg][c * 8 + e] = mn[e];
+  }
+  __syncthreads();
+  for (int d = t; d < D; d += kThreads) {
+    double sacc = 0.0;
+    float a = -INFINITY, z = INFINITY;
+    for (int g = 0; g < RG; ++g) {
+      sacc += red[g][d];
+      a = fmaxf(a, redmx[g][d]);
+      z = fminf(z, redmn[g][d]);
+    }
+    sum[d] = sacc;
+    if (extremes) {
+      cmax[d] = a;
+      cmin[d] = z;
+    }
+  }
+}
+
 // grid (nsplit, Hq, B): chunk `split` of sequence b, head h.
-//   K (h < Hkv): ksum[bh, split, d] = sum over the chunk's tokens, binary64; with a
-//     second-level scale also kmax / kmin per channel.
-//   Q (h < Hq) and V (h < Hkv), second-level scale only: max |x| over the chunk.
+//   K (h < Hkv, K smoothing or a second-level scale): ksum[bh, split, d] = sum over the
+//     chunk's tokens, binary64; with a second-level scale also kmax / kmin per channel.
+//   Q (h < Hq, Q smoothing): the same statistics of Q into qsum / qmax / qmin.
+//   Q without smoothing (h < Hq) and V (h < Hkv), second-level scale only: max |x| over
+//   the chunk.
 template <int D>
 __global__ void __launch_bounds__(kThreads) stats_kernel(QuantParams p) {
   constexpr int CPR = D / 8;          // 16-byte chunks per row
@@ -204,51 +259,20 @@ __global__ void __launch_bounds__(kThreads) stats_kernel(QuantParams p) {
   const int n0 = split * kChunk;
 
   if (h < p.Hkv && (p.smooth_k || gs) && n0 < si.len_k) {
-    const int n1 = min(n0 + kChunk, si.len_k);
-    double acc[8];
-    float mx[8], mn[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      acc[e] = 0.0;
-      mx[e] = -INFINITY;
-      mn[e] = INFINITY;
-    }
-#pragma unroll 4
-    for (int n = n0 + rg; n < n1; n += RG) {
-      float x[8];
-      unpack8(ld_nc_16(row_ptr(p.k, p.sk, b, h, static_cast<int64_t>(si.tok_k) + n) + c * 16), p.dtype, x);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        acc[e] += static_cast<double>(x[e]);
-        mx[e] = fmaxf(mx[e], x[e]);
-        mn[e] = fminf(mn[e], x[e]);
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      red[rg][c * 8 + e] = acc[e];
-      redmx[rg][c * 8 + e] = mx[e];
-      redmn[rg][c * 8 + e] = mn[e];
-    }
-    __syncthreads();
     const size_t base = (static_cast<size_t>(b * p.Hkv + h) * p.nsplit + split) * D;
-    for (int d = t; d < D; d += kThreads) {
-      double s = 0.0;
-      float a = -INFINITY, z = INFINITY;
-      for (int g = 0; g < RG; ++g) {
-        s += red[g][d];
-        a = fmaxf(a, redmx[g][d]);
-        z = fminf(z, redmn[g][d]);
-      }
-      p.ksum[base + d] = s;
-      if (gs) {
-        p.kmax[base + d] = a;
-        p.kmin[base + d] = z;
-      }
-    }
+    chunk_channel_stats<D>(p.k, p.sk, p.dtype, b, h, si.tok_k, n0, min(n0 + kChunk, si.len_k), gs,
+                           p.ksum + base, gs ? p.kmax + base : nullptr, gs ? p.kmin + base : nullptr,
+                           red, redmx, redmn);
+  }
+  if (h < p.Hq && p.smooth_q && n0 < si.len_q) {
+    const size_t base = (static_cast<size_t>(b * p.Hq + h) * p.nsplit + split) * D;
+    chunk_channel_stats<D>(p.q, p.sq, p.dtype, b, h, si.tok_q, n0, min(n0 + kChunk, si.len_q), gs,
+                           p.qsum + base, gs ? p.qmax + base : nullptr, gs ? p.qmin + base : nullptr,
+                           red, redmx, redmn);
   }
   if (!gs) return;
-  for (int job = 0; job < 2; ++job) {  // 0: Q, 1: V
+  for (int job = 0; job < 2; ++job) {  // 0: Q (unsmoothed), 1: V
+    if (job == 0 && p.smooth_q) continue;
     const int H = job == 0 ? p.Hq : p.Hkv;
     const int len = job == 0 ? si.len_q : si.len_k;
     if (h >= H || n0 >= len) continue;
@@ -257,6 +281,7 @@ __global__ void __launch_bounds__(kThreads) stats_kernel(QuantParams p) {
     const Strides& st = job == 0 ? p.sq : p.sv;
     const int tok = job == 0 ? si.tok_q : si.tok_k;
     float a = 0.0f;
+#pragma unroll 4
     for (int n = n0 + rg; n < n1; n += RG) {
       float x[8];
       unpack8(ld_nc_16(row_ptr(src, st, b, h, static_cast<int64_t>(tok) + n) + c * 16), p.dtype, x);
@@ -268,8 +293,9 @@ __global__ void __launch_bounds__(kThreads) stats_kernel(QuantParams p) {
   }
 }
 
-// grid (Hq, B), D threads: the K mean of (sequence b, key/value head h) and the
-// second-level maxima of Q (head h) and of K - mean and V (head h).
+// grid (Hq, B), D threads: the K mean of (sequence b, key/value head h), the Q mean of
+// query head h (Q smoothing), and the second-level maxima of Q (or Q - mean) for head h
+// and of K - mean and V for head h.
 template <int D>
 __global__ void __launch_bounds__(D) finalize_kernel(QuantParams p) {
   __shared__ float redw[D / 32];
@@ -306,12 +332,34 @@ __global__ void __launch_bounds__(D) finalize_kernel(QuantParams p) {
       }
     }
   }
-  if (gs && h < p.Hq) {
+  if (h < p.Hq && (gs || p.smooth_q)) {
     const int ns = (si.len_q + kChunk - 1) / kChunk;
     float aq = 0.0f;
-    for (int g = d; g < ns; g += D) aq = fmaxf(aq, p.qamax[static_cast<size_t>(b * p.Hq + h) * p.nsplit + g]);
-    aq = block_max(aq, redw);
-    if (d == 0) amax_store(p.amax + (p.gscale == kGscaleHead ? b * p.Hq + h : 0), p.gscale, aq);
+    if (p.smooth_q) {
+      // The query mean, and (second-level scale) the maximum of |fp32(q - mu_q)|.
+      const size_t base = static_cast<size_t>(b * p.Hq + h) * p.nsplit * D + d;
+      float mu = 0.0f;
+      if (si.len_q > 0) {
+        double s = 0.0;
+        for (int g = 0; g < ns; ++g) s += p.qsum[base + static_cast<size_t>(g) * D];
+        mu = static_cast<float>(s / static_cast<double>(si.len_q));
+      }
+      p.q_mean[static_cast<size_t>(b * p.Hq + h) * D + d] = mu;
+      if (gs && si.len_q > 0) {
+        float mx = -INFINITY, mn = INFINITY;
+        for (int g = 0; g < ns; ++g) {
+          mx = fmaxf(mx, p.qmax[base + static_cast<size_t>(g) * D]);
+          mn = fminf(mn, p.qmin[base + static_cast<size_t>(g) * D]);
+        }
+        aq = fmaxf(fabsf(__fsub_rn(mx, mu)), fabsf(__fsub_rn(mn, mu)));
+      }
+    } else {
+      for (int g = d; g < ns; g += D) aq = fmaxf(aq, p.qamax[static_cast<size_t>(b * p.Hq + h) * p.nsplit + g]);
+    }
+    if (gs) {
+      aq = block_max(aq, redw);
+      if (d == 0) amax_store(p.amax + (p.gscale == kGscaleHead ? b * p.Hq + h : 0), p.gscale, aq);
+    }
   }
 }
 
@@ -345,9 +393,9 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
   if (job < 2) {
     uint8_t* sfbuf = smem;                                  // kSfBytesQK
     float* mu = reinterpret_cast<float*>(smem + 1024);      // D floats
-    const bool smooth = (job == 1) && p.smooth_k;
-    for (int d = t; d < D; d += kThreads)
-      mu[d] = smooth ? p.k_mean[static_cast<size_t>(b * p.Hkv + h) * D + d] : 0.0f;
+    const bool smooth = (job == 1) ? p.smooth_k != 0 : p.smooth_q != 0;
+    const float* mean_src = (job == 1 ? p.k_mean : p.q_mean) + static_cast<size_t>(b * H + h) * D;
+    for (int d = t; d < D; d += kThreads) mu[d] = smooth ? mean_src[d] : 0.0f;
     for (int i = t; i < kSfBytesQK / 16; i += kThreads) reinterpret_cast<uint4*>(sfbuf)[i] = make_uint4(0, 0, 0, 0);
     __syncthreads();
     const void* src = job == 0 ? p.q : p.k;
@@ -371,15 +419,54 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
       const int rl = rl0 + it * kRowStep;
       float x[8];
       unpack8(raw[it], p.dtype, x);
-      if (rl < rows) {
-        if (smooth) {
+      if (rl < rows && smooth) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], m8[e]);
-        }
-        if (gs) {
+        for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], m8[e]);
+      }
+      if (job == 1 && p.smooth_q) {
+        // Q smoothing bias of this key for every query head of the group:
+        // mu_q . (k - mu_k), over the CPR lanes that hold the row (zero for padding).
+        const int G = p.Hq / p.Hkv;
+        for (int gi = 0; gi < G; ++gi) {
+          const int hq = h * G + gi;
+          const float4* mq = reinterpret_cast<const float4*>(p.q_mean + static_cast<size_t>(b * p.Hq + hq) * D + c * 8);
+          const float4 m0 = mq[0], m1 = mq[1];
+          float acc = x[0] * m0.x;
+          acc = fmaf(x[1], m0.y, acc);
+          acc = fmaf(x[2], m0.z, acc);
+          acc = fmaf(x[3], m0.w, acc);
+          acc = fmaf(x[4], m1.x, acc);
+          acc = fmaf(x[5], m1.y, acc);
+          acc = fmaf(x[6], m1.z, acc);
+          acc = fmaf(x[7], m1.w, acc);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = __fdiv_rn(x[e], g);
+          for (int o = CPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          if (c == 0) {
+            if (gs) {
+              const float gq = second_level_scale(p.amax[p.gscale == kGscaleHead ? b * p.Hq + hq : 0]);
+              acc = __fdiv_rn(acc, gq * g);
+            }
+            // Three bf16 terms (their sum is acc to about 2^-24 relative) in the operand
+            // layout the attention kernel's bias MMA reads: 8-key groups of 256 bytes, two
+            // 128-byte halves of 8 keys x 16 bytes.
+            const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
+            const float r1 = acc - __bfloat162float(hi);
+            const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+            const uint32_t w0 = static_cast<uint32_t>(__bfloat16_as_ushort(hi)) |
+                                (static_cast<uint32_t>(__bfloat16_as_ushort(mid)) << 16);
+            const uint32_t w1 = static_cast<uint32_t>(__bfloat16_as_ushort(lo));
+            uint8_t* tb = p.qk_bias + (static_cast<int64_t>(p.Hq) * prow + static_cast<int64_t>(hq) * ntile * 128 +
+                                       tile * 128) * 32;
+            uint8_t* row = tb + (rl >> 3) * 256 + (rl & 7) * 16;
+            *reinterpret_cast<uint4*>(row) = make_uint4(w0, w1, 0u, 0u);
+            *reinterpret_cast<uint4*>(row + 128) = make_uint4(0u, 0u, 0u, 0u);
+          }
         }
+      }
+      if (rl < rows && gs) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = __fdiv_rn(x[e], g);
       }
       float a = 0.0f;
 #pragma unroll
@@ -464,7 +551,7 @@ cudaError_t launch_quantize(const QuantParams& p, const QuantLaunch& l, cudaStre
     if (e != cudaSuccess) return e;
   }
   const bool gs = p.gscale != kGscaleNone;
-  if ((p.smooth_k || gs) && p.nsplit > 0) {
+  if ((p.smooth_k || p.smooth_q || gs) && p.nsplit > 0) {
     dim3 g1(p.nsplit, p.Hq, p.B);
     if (p.D == 64) stats_kernel<64><<<g1, kThreads, 0, stream>>>(p);
     else stats_kernel<128><<<g1, kThreads, 0, stream>>>(p);
@@ -472,7 +559,7 @@ cudaError_t launch_quantize(const QuantParams& p, const QuantLaunch& l, cudaStre
     if (e != cudaSuccess) return e;
   }
   // The finalize pass writes the K mean (zeros without smoothing) and the maxima.
-  if (p.k_mean != nullptr || gs) {
+  if (p.k_mean != nullptr || gs || p.smooth_q) {
     dim3 g2(p.Hq, p.B);
     if (p.D == 64) finalize_kernel<64><<<g2, 64, 0, stream>>>(p);
     else finalize_kernel<128><<<g2, 128, 0, stream>>>(p);

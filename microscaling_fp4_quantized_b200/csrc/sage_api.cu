@@ -92,7 +92,7 @@ size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 // A checked problem with everything derived from it.
 struct Prob {
   sage_fp4_problem_t u;  // the caller's description (sm_scale resolved)
-  bool packed, empty, gs;
+  bool packed, empty, gs, sq;
   int64_t rows_q, rows_k;  // padded token rows per head (packed: an upper bound)
   int tiles_q, tiles_k, nsplit;
 };
@@ -117,6 +117,7 @@ sage_status_t check_problem(const sage_fp4_problem_t* in, Prob* p) {
     p->u.q_stride[0] = p->u.k_stride[0] = p->u.v_stride[0] = p->u.o_stride[0] = 0;
   }
   p->gs = u.gscale != SAGE_GSCALE_NONE;
+  p->sq = u.smooth_q != 0;
   const int64_t* strides[4] = {p->u.q_stride, p->u.k_stride, p->u.v_stride, p->u.o_stride};
   for (const int64_t* s : strides)
     for (int i = 0; i < 3; ++i)
@@ -161,15 +162,20 @@ sage_fp4_problem_sizes_t sizes_of(const Prob& p) {
   z.k_mean = static_cast<size_t>(B * Hkv * D * 4);
   z.amax = static_cast<size_t>(3 * B * Hq * 4);
   z.seq = p.packed ? static_cast<size_t>((2 * (B + 1) + 4) * 4) : 0;
+  z.q_mean = p.sq ? static_cast<size_t>(B * Hq * D * 4) : 0;
+  z.qk_bias = p.sq ? static_cast<size_t>(Hq * p.rows_k * 32) : 0;
   const int64_t ns = p.nsplit;
   size_t scratch = 0;
-  if (p.u.smooth_k || p.gs) scratch += up256(static_cast<size_t>(B * Hkv * ns * D * 8));
+  if (p.u.smooth_k || p.gs || p.sq) scratch += up256(static_cast<size_t>(B * Hkv * ns * D * 8));
   if (p.gs)
     scratch += 2 * up256(static_cast<size_t>(B * Hkv * ns * D * 4)) + up256(static_cast<size_t>(B * Hq * ns * 4)) +
                up256(static_cast<size_t>(B * Hkv * ns * 4));
+  if (p.sq) scratch += up256(static_cast<size_t>(B * Hq * ns * D * 8));
+  if (p.sq && p.gs) scratch += 2 * up256(static_cast<size_t>(B * Hq * ns * D * 4));
   z.scratch = scratch;
   z.workspace = up256(z.q_fp4) + up256(z.q_sf) + up256(z.k_fp4) + up256(z.k_sf) + up256(z.vt_fp4) +
-                up256(z.vt_sf) + up256(z.k_mean) + up256(z.amax) + up256(z.seq) + z.scratch;
+                up256(z.vt_sf) + up256(z.k_mean) + up256(z.amax) + up256(z.seq) + up256(z.q_mean) +
+                up256(z.qk_bias) + z.scratch;
   return z;
 }
 
@@ -188,6 +194,8 @@ void carve(const Prob& p, void* base, sage_fp4_quantized_t* qz, void** scratch) 
   qz->k_mean = reinterpret_cast<float*>(take(z.k_mean));
   qz->amax = reinterpret_cast<float*>(take(z.amax));
   qz->seq = p.packed ? reinterpret_cast<int32_t*>(take(z.seq)) : nullptr;
+  qz->q_mean = p.sq ? reinterpret_cast<float*>(take(z.q_mean)) : nullptr;
+  qz->qk_bias = p.sq ? take(z.qk_bias) : nullptr;
   *scratch = z.scratch ? b + off : nullptr;
 }
 
@@ -218,6 +226,8 @@ sage_status_t check_bundle(const Prob& p, const sage_fp4_quantized_t* qz, bool n
   if (need_kmean && (qz->k_mean == nullptr || !aligned16(qz->k_mean))) return SAGE_ERR_INVALID_ARG;
   if (p.gs && (qz->amax == nullptr || !aligned16(qz->amax))) return SAGE_ERR_INVALID_ARG;
   if (p.packed && (qz->seq == nullptr || !aligned16(qz->seq))) return SAGE_ERR_INVALID_ARG;
+  if (p.sq && (qz->qk_bias == nullptr || !aligned16(qz->qk_bias))) return SAGE_ERR_INVALID_ARG;
+  if (p.sq && need_kmean && (qz->q_mean == nullptr || !aligned16(qz->q_mean))) return SAGE_ERR_INVALID_ARG;
   return SAGE_OK;
 }
 
@@ -240,6 +250,9 @@ sage_status_t run_quantize(const Prob& p, const void* q, const void* k, const vo
   k_.D = p.u.D;
   k_.seq = seq_map(p, qz);
   k_.smooth_k = p.u.smooth_k ? 1 : 0;
+  k_.smooth_q = p.sq ? 1 : 0;
+  k_.q_mean = p.sq ? qz.q_mean : nullptr;
+  k_.qk_bias = p.sq ? qz.qk_bias : nullptr;
   k_.gscale = p.u.gscale;
   k_.nsplit = p.nsplit;
   k_.amax_stride = p.u.B * p.u.Hq;
@@ -254,12 +267,17 @@ sage_status_t run_quantize(const Prob& p, const void* q, const void* k, const vo
   const int64_t B = p.u.B, Hq = p.u.Hq, Hkv = p.u.Hkv, ns = p.nsplit, D = p.u.D;
   uint8_t* s = static_cast<uint8_t*>(scratch);
   auto take = [&](size_t n) { uint8_t* r = s; s += up256(n); return r; };
-  if (p.u.smooth_k || p.gs) k_.ksum = reinterpret_cast<double*>(take(static_cast<size_t>(B * Hkv * ns * D * 8)));
+  if (p.u.smooth_k || p.gs || p.sq) k_.ksum = reinterpret_cast<double*>(take(static_cast<size_t>(B * Hkv * ns * D * 8)));
   if (p.gs) {
     k_.kmax = reinterpret_cast<float*>(take(static_cast<size_t>(B * Hkv * ns * D * 4)));
     k_.kmin = reinterpret_cast<float*>(take(static_cast<size_t>(B * Hkv * ns * D * 4)));
     k_.qamax = reinterpret_cast<float*>(take(static_cast<size_t>(B * Hq * ns * 4)));
     k_.vamax = reinterpret_cast<float*>(take(static_cast<size_t>(B * Hkv * ns * 4)));
+  }
+  if (p.sq) k_.qsum = reinterpret_cast<double*>(take(static_cast<size_t>(B * Hq * ns * D * 8)));
+  if (p.sq && p.gs) {
+    k_.qmax = reinterpret_cast<float*>(take(static_cast<size_t>(B * Hq * ns * D * 4)));
+    k_.qmin = reinterpret_cast<float*>(take(static_cast<size_t>(B * Hq * ns * D * 4)));
   }
   if (p.packed) {
     k_.total_q = p.u.total_q;
@@ -317,6 +335,7 @@ sage_status_t run_attention(const Prob& p, const sage_fp4_quantized_t& qz, void*
   a.group = p.u.Hq / p.u.Hkv;
   a.seq = seq_map(p, qz);
   a.amax = p.gs ? qz.amax : nullptr;
+  a.qk_bias = p.sq ? qz.qk_bias : nullptr;
   a.gscale = p.u.gscale;
   a.amax_stride = p.u.B * p.u.Hq;
   return cuda_status(sage::launch_attention(m, a, p.tiles_q, stream));

@@ -89,6 +89,7 @@ struct QuantParams {
   int B, Hq, Hkv, D;
   SeqMap seq;
   int smooth_k;
+  int smooth_q;      // subtract the per-(sequence, head) query mean; emit the per-key bias
   int gscale;
   int nsplit;        // 512-token chunks of the longest sequence
   int amax_stride;   // B * Hq: distance between the Q, K and V maxima
@@ -99,10 +100,16 @@ struct QuantParams {
   uint8_t* vt_fp4;
   uint8_t* vt_sf;
   float* k_mean;     // [B * Hkv, D]
+  float* q_mean;     // [B * Hq, D]              (smooth_q)
+  uint8_t* qk_bias;  // (smooth_q) per (query head, padded key row) 32 bytes: the bias
+                     // mu_q . (k - mu_k) / (g_q g_k) as three bf16 terms, MMA operand layout
   float* amax;       // [3, B * Hq]; tensor mode uses element 0 of each
   double* ksum;      // [B * Hkv, nsplit, D]
   float* kmax;       // [B * Hkv, nsplit, D]  (second-level scale only)
   float* kmin;       // [B * Hkv, nsplit, D]
+  double* qsum;      // [B * Hq, nsplit, D]   (smooth_q)
+  float* qmax;       // [B * Hq, nsplit, D]   (smooth_q with a second-level scale)
+  float* qmin;       // [B * Hq, nsplit, D]
   float* qamax;      // [B * Hq, nsplit]
   float* vamax;      // [B * Hkv, nsplit]
   // Packed problems: the plan kernel's inputs and outputs.
@@ -124,6 +131,7 @@ struct AttnParams {
   int B, Hq, Hkv, group, D;
   SeqMap seq;
   const float* amax;    // second-level maxima, or nullptr
+  const uint8_t* qk_bias; // Q-smoothing bias operand per (query head, padded key row), or nullptr
   int gscale;
   int amax_stride;
   int BH, Np;           // dense S = Q^ K^^T (scores kernel only)

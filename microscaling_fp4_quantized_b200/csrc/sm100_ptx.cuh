@@ -155,6 +155,19 @@ __device__ __forceinline__ void tc_mma_fp4(uint32_t d_tmem, uint64_t adesc, uint
       : "memory");
 }
 
+// D (FP32, TMEM) += A B^T for bf16 A [M x K] and B [N x K] in shared memory (kind::f16,
+// one instruction covers K = 16).
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Each thread of the warp reads 32 consecutive 32-bit columns of its own lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -245,6 +258,16 @@ __host__ __device__ constexpr uint32_t make_idesc_fp4(uint32_t n) {
          | (1u << 10)              // B format: E2M1
          | ((n >> 3) << 17)        // N / 8
          | (0u << 23)              // scale format: UE4M3
+         | ((128u >> 4) << 24);    // M / 16
+}
+
+// Instruction descriptor for kind::f16 with bf16 A/B, an FP32 accumulator, K-major A and
+// B, dense, M = 128 and the given N.
+__host__ __device__ constexpr uint32_t make_idesc_bf16(uint32_t n) {
+  return (1u << 4)                 // D format: F32
+         | (1u << 7)               // A format: BF16
+         | (1u << 10)              // B format: BF16
+         | ((n >> 3) << 17)        // N / 8
          | ((128u >> 4) << 24);    // M / 16
 }
 

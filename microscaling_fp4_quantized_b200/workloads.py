@@ -121,7 +121,9 @@ def make_inputs(w: Workload, device: Optional[str] = None):
 # Recipe: one CPU generator seeded with the workload's seed draws, in this order,
 # Q [Tq, Hq, D], K [Tk, Hkv, D], V [Tk, Hkv, D] ~ N(0, 1) in float32 (Tq, Tk = the summed
 # lengths; sequence b owns the next lens[b] tokens), then one K bias per (sequence, key
-# head) ~ N(0, sigma^2) [B, Hkv, D] added to that sequence's keys. Q, K and V are then
+# head) ~ N(0, sigma^2) [B, Hkv, D] added to that sequence's keys, then (only when
+# q_bias_sigma > 0) one query offset per (sequence, query head) ~ N(0, q_bias_sigma^2)
+# [B, Hq, D] added to that sequence's queries. Q, K and V are then
 # multiplied by q_scale, k_scale and v_scale (to reach the one-level format's range
 # limits) and cast to the dtype. Dense workloads view the same draws as [B, H, N, D]
 # ("HND") or [B, N, H, D] ("NHD") tensors.
@@ -144,6 +146,8 @@ class GeneralWorkload:
     k_scale: float = 1.0
     v_scale: float = 1.0
     gscale: str = "none"
+    smooth_q: bool = False
+    q_bias_sigma: float = 0.0
 
     @property
     def B(self) -> int:
@@ -166,7 +170,7 @@ class GeneralWorkload:
                 "total_q": sum(self.lens_q), "total_k": sum(self.lens_k), "causal": self.causal,
                 "packed": self.packed, "layout": self.layout,
                 "dtype": str(self.dtype).replace("torch.", ""), "seed": self.seed,
-                "gscale": self.gscale}
+                "gscale": self.gscale, "smooth_q": self.smooth_q, "q_bias_sigma": self.q_bias_sigma}
 
 
 def general(name: str, Hq: int, Hkv: int, D: int, lens_q, lens_k=None, causal: bool = False,
@@ -204,6 +208,10 @@ def make_general_inputs(w: GeneralWorkload, device: Optional[str] = None) -> dic
     cu_k = torch.tensor([0] + list(itertools.accumulate(w.lens_k)), dtype=torch.int32)
     for b in range(w.B):
         k[cu_k[b]:cu_k[b + 1]] += bias[b]
+    if w.q_bias_sigma > 0:
+        qbias = torch.randn((w.B, w.Hq, w.D), generator=g, dtype=torch.float32) * w.q_bias_sigma
+        for b in range(w.B):
+            q[cu_q[b]:cu_q[b + 1]] += qbias[b]
     q, k, v = (q * w.q_scale).to(w.dtype), (k * w.k_scale).to(w.dtype), (v * w.v_scale).to(w.dtype)
     out = {"cu_seqlens_q": cu_q, "cu_seqlens_k": cu_k}
     if w.packed:

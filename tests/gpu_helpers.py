@@ -78,6 +78,19 @@ def _sf_rows(sf: np.ndarray, rows: np.ndarray, D: int) -> np.ndarray:
     return sf[idx]
 
 
+def decode_bias(buf: np.ndarray, row0: int, n: int) -> np.ndarray:
+    """Sum of the three bf16 terms of keys 0..n-1 of the bias operand starting at padded
+    row row0 (a multiple of 128) -> float64 [n]."""
+    keys = np.arange(n)
+    tile = row0 + (keys // 128) * 128
+    k = keys % 128
+    off = tile * 32 + (k // 8) * 256 + (k % 8) * 16
+    words = np.stack([buf[off + 2 * i].astype(np.uint16) | (buf[off + 2 * i + 1].astype(np.uint16) << 8)
+                      for i in range(3)])
+    vals = (words.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return vals.sum(axis=0)
+
+
 def canonical_problem(qz: dict, lens_q, lens_k, Hq: int, Hkv: int, D: int) -> list:
     """Per sequence, the GPU's quantized tensors of a general problem in the oracle's
     canonical layouts: q_codes [Hq, Lq, D/2], q_sf [Hq, Lq, D/16], k_codes / k_sf
@@ -85,6 +98,8 @@ def canonical_problem(qz: dict, lens_q, lens_k, Hq: int, Hkv: int, D: int) -> li
     k_mean [Hkv, D]; plus pads_zero (the padding rows and tokens hold zeros)."""
     g = {k: qz[k].cpu().numpy() for k in ("q_fp4", "q_sf", "k_fp4", "k_sf", "vt_fp4", "vt_sf")}
     kmean = qz["k_mean"].cpu().numpy()
+    qmean = qz["q_mean"].cpu().numpy() if "q_mean" in qz else None
+    bias = qz["qk_bias"].cpu().numpy() if "qk_bias" in qz else None
     pq, pk = padded_offsets(lens_q), padded_offsets(lens_k)
     res = []
     for b, (Lq, Lk) in enumerate(zip(lens_q, lens_k)):
@@ -121,6 +136,12 @@ def canonical_problem(qz: dict, lens_q, lens_k, Hq: int, Hkv: int, D: int) -> li
         o["k_codes"], o["k_sf"] = np.stack(kc), np.stack(ks)
         o["vt_codes"], o["vt_sf"] = np.stack(vc), np.stack(vs)
         o["k_mean"] = kmean[b * Hkv * D:(b + 1) * Hkv * D].reshape(Hkv, D)
+        if qmean is not None and qmean.size >= (b + 1) * Hq * D:
+            o["q_mean"] = qmean[b * Hq * D:(b + 1) * Hq * D].reshape(Hq, D)
+        if bias is not None and bias.size >= 32 * Hq * (pk[b] + Pk):
+            # the Q-smoothing bias operand: 32 bytes per (query head, padded key row), three
+            # bf16 terms in elements 0-2, key n of a tile at (n/8)*256 + (n%8)*16
+            o["qk_bias"] = np.stack([decode_bias(bias, Hq * pk[b] + h * Pk, Lk) for h in range(Hq)])
         res.append(o)
     return res
 

@@ -2,10 +2,12 @@
 query and key lengths that differ (causal mask aligned to the last key), packed
 variable-length sequences, and the second-level (per-tensor / per-head) scales.
 
-Quantization: K mean within 1 ulp, second-level maxima exact, codes and scale bytes bit
-for bit against the oracle fed the GPU's K mean. Attention: the bar of the dense tests
-(max |O_gpu - O_oracle| <= 1e-2 * max|V| and cosine >= 0.999 against the oracle's
-emulation with the same key-tile width, 128), per sequence.
+Quantization: K and Q means within 1 ulp, second-level maxima exact, codes and scale
+bytes bit for bit against the oracle fed the GPU's means, Q-smoothing bias within 1e-5
+relative. Attention: the bar of the dense tests (max |O_gpu - O_oracle| <= 1e-2 * max|V|
+and cosine >= 0.999 against the oracle's emulation with the same key-tile width, 128),
+per sequence; a row over the max-abs bar is accepted only as a rare, valid alternative
+result (see _check_rows_over_bar).
 """
 import numpy as np
 import pytest
@@ -60,26 +62,30 @@ def _out_per_seq(w, x, out):
 def _problem(sage, w, x, out):
     if w.packed:
         return sage.sageattn_varlen_problem(x["q"], x["k"], x["v"], out, x["cu_seqlens_q"], x["cu_seqlens_k"],
-                                            max(w.lens_q), max(w.lens_k), w.causal, None, True, w.gscale)
-    return sage.sageattn_problem(x["q"], x["k"], x["v"], out, w.layout, w.causal, None, True, w.gscale)
+                                            max(w.lens_q), max(w.lens_k), w.causal, None, True, w.gscale,
+                                            w.smooth_q)
+    return sage.sageattn_problem(x["q"], x["k"], x["v"], out, w.layout, w.causal, None, True, w.gscale,
+                                 w.smooth_q)
 
 
-def _run(sage, w, x, gscale=None):
+def _run(sage, w, x, gscale=None, smooth_q=None):
     g = w.gscale if gscale is None else gscale
+    sq = w.smooth_q if smooth_q is None else smooth_q
     if w.packed:
         return sage.sageattn_varlen(x["q"], x["k"], x["v"], x["cu_seqlens_q"], x["cu_seqlens_k"],
-                                    max(w.lens_q), max(w.lens_k), is_causal=w.causal, gscale=g)
-    return sage.sageattn(x["q"], x["k"], x["v"], tensor_layout=w.layout, is_causal=w.causal, gscale=g)
+                                    max(w.lens_q), max(w.lens_k), is_causal=w.causal, gscale=g, smooth_q=sq)
+    return sage.sageattn(x["q"], x["k"], x["v"], tensor_layout=w.layout, is_causal=w.causal, gscale=g,
+                         smooth_q=sq)
 
 
-def _oracle_amax(oracle_mod, w, seqs, kmeans):
+def _oracle_amax(oracle_mod, w, seqs, kmeans, qmeans):
     """Second-level maxima the library must reproduce exactly (tensor mode: over all)."""
     if w.gscale != "tensor":
         return [None] * len(seqs)
     a = {"q": 0.0, "k": 0.0, "v": 0.0}
-    for (qs, ks, vs), km in zip(seqs, kmeans):
+    for (qs, ks, vs), km, qm in zip(seqs, kmeans, qmeans):
         if qs.shape[1]:
-            a["q"] = max(a["q"], float(oracle_mod.group_amax(qs).max()))
+            a["q"] = max(a["q"], float(oracle_mod.group_amax(qs, qm).max()))
         if ks.shape[1]:
             a["k"] = max(a["k"], float(oracle_mod.group_amax(ks, km).max()))
             a["v"] = max(a["v"], float(oracle_mod.group_amax(vs).max()))
@@ -96,6 +102,12 @@ QUANT_CASES = [
               q_scale=1e-3, v_scale=4000.0),
     W.general("packed_cross_lengths", 2, 1, 64, (100, 37, 513, 0), (300, 37, 129, 50), causal=True, seed=55,
               gscale="tensor"),
+    W.general("qsmooth_gqa_dense", 8, 2, 128, (700, 700), causal=True, packed=False, seed=56, smooth_q=True,
+              q_bias_sigma=4.0),
+    W.general("qsmooth_packed_tensor_scale", 4, 2, 64, (5, 0, 300, 128, 1, 1000), seed=57, smooth_q=True,
+              gscale="tensor", q_bias_sigma=3.0),
+    W.general("qsmooth_cross_head_scale", 4, 4, 128, (200,), (600,), causal=True, packed=False, seed=58,
+              smooth_q=True, gscale="head", q_bias_sigma=2.0, v_scale=3000.0),
 ]
 
 
@@ -109,7 +121,8 @@ def test_general_quant_bit_exact(sage, oracle_mod, w):
     can = canonical_problem(qz, w.lens_q, w.lens_k, w.Hq, w.Hkv, w.D)
     seqs = _per_seq(w, x)
     kmeans = [c["k_mean"] for c in can]
-    amax_t = _oracle_amax(oracle_mod, w, seqs, kmeans)
+    qmeans = [c.get("q_mean") for c in can]
+    amax_t = _oracle_amax(oracle_mod, w, seqs, kmeans, qmeans)
     amax_gpu = qz["amax"].cpu().numpy()[: 3 * w.B * w.Hq].reshape(3, w.B * w.Hq)
     for b, ((qs, ks, vs), c) in enumerate(zip(seqs, can)):
         assert c["pads_zero"], f"sequence {b}: padding not zero"
@@ -117,10 +130,22 @@ def test_general_quant_bit_exact(sage, oracle_mod, w):
             km = oracle_mod.kmean(ks)
             ulp = np.abs(c["k_mean"].view(np.int32).astype(np.int64) - km.view(np.int32).astype(np.int64))
             assert ulp.max() <= 1, f"sequence {b}: K mean differs by {ulp.max()} ulp"
+        if w.smooth_q and qs.shape[1]:
+            qm = oracle_mod.kmean(qs)
+            ulp = np.abs(c["q_mean"].view(np.int32).astype(np.int64) - qm.view(np.int32).astype(np.int64))
+            assert ulp.max() <= 1, f"sequence {b}: Q mean differs by {ulp.max()} ulp"
         if qs.shape[1] == 0 and ks.shape[1] == 0:
             continue
         o = oracle_mod.quantize_qkv(qs, ks, vs, smooth_k=True, kmean_in=c["k_mean"], gscale=w.gscale,
-                                    amax_in=amax_t[b], heads=(1, w.Hq, w.Hkv))
+                                    amax_in=amax_t[b], heads=(1, w.Hq, w.Hkv), smooth_q=w.smooth_q,
+                                    qmean_in=c.get("q_mean") if w.smooth_q else None)
+        if w.smooth_q and ks.shape[1]:
+            want = o["qk_bias"]
+            if w.gscale != "none":
+                gk = np.repeat(o["gk"], w.Hq // w.Hkv)
+                want = want / (o["gq"].astype(np.float64) * gk)[:, None]
+            err = np.max(np.abs(c["qk_bias"] - want)) / max(np.max(np.abs(want)), 1e-30)
+            assert err <= 1e-5, f"sequence {b}: Q-smoothing bias relative error {err}"
         if w.gscale == "head":
             assert np.array_equal(amax_gpu[0, b * w.Hq:(b + 1) * w.Hq], o["amax"]["q"]) or qs.shape[1] == 0
             if ks.shape[1]:
@@ -146,6 +171,26 @@ ATTN_CASES = QUANT_CASES + [
 ]
 
 
+def _check_rows_over_bar(oracle_mod, w, qs, ks, vs, g, e, rows, tol, b):
+    """Rows whose max-abs difference from the emulation exceeds the bar. P^ codes are not
+    unique (the GPU's FP32 scores round differently from the oracle's binary64 ones), and
+    when attention is strongly peaked one code that flips at a rounding boundary on a
+    dominant key moves that row by a few percent of |V|. Such a row is accepted only if it
+    is rare (at most 0.1 % of the rows, one at least) and it is as close to exact
+    attention as the emulated row is, within the same bar."""
+    Lq = qs.shape[1]
+    if rows is None:
+        rows = np.array([(h, i) for h in range(w.Hq) for i in range(Lq)], np.int64)
+    err = np.abs(g - e).max(axis=1)
+    over = np.flatnonzero(err > tol)
+    assert len(over) <= max(1, len(err) // 1000), (b, len(over), float(err.max()), tol)
+    if len(over):
+        ex = oracle_mod.attn_exact(qs, ks, vs, w.causal, w.sm_scale, rows=rows[over], heads=(1, w.Hq, w.Hkv))
+        d_gpu = np.abs(g[over] - ex).max(axis=1)
+        d_emu = np.abs(e[over] - ex).max(axis=1)
+        assert (d_gpu <= d_emu + tol).all(), (b, rows[over].tolist(), d_gpu.tolist(), d_emu.tolist(), tol)
+
+
 def _check_attention(sage, oracle_mod, w, rows_per_seq=None):
     x = W.make_general_inputs(w, "cuda")
     out = _run(sage, w, x)
@@ -155,9 +200,11 @@ def _check_attention(sage, oracle_mod, w, rows_per_seq=None):
     # The GPU's K means (bit-exact quantization is checked separately) feed the oracle.
     qz = sage.quantize(_problem(sage, w, x, torch.empty_like(out)), x["q"], x["k"], x["v"])
     torch.cuda.synchronize()
-    kmeans = [c["k_mean"] for c in canonical_problem(qz, w.lens_q, w.lens_k, w.Hq, w.Hkv, w.D)]
+    can = canonical_problem(qz, w.lens_q, w.lens_k, w.Hq, w.Hkv, w.D)
+    kmeans = [c["k_mean"] for c in can]
+    qmeans = [c.get("q_mean") for c in can]
     seqs = _per_seq(w, x)
-    amax_t = _oracle_amax(oracle_mod, w, seqs, kmeans)
+    amax_t = _oracle_amax(oracle_mod, w, seqs, kmeans, qmeans)
     worst = None
     for b, ((qs, ks, vs), got) in enumerate(zip(seqs, got_all)):
         Lq = qs.shape[1]
@@ -175,12 +222,15 @@ def _check_attention(sage, oracle_mod, w, rows_per_seq=None):
             rows = np.array([(h, i) for h in heads for i in rr], np.int64)
         em, _ = oracle_mod.attention(qs, ks, vs, w.causal, w.sm_scale, Bk=BK, rows=rows,
                                      kmean_in=kmeans[b], gscale=w.gscale, heads=(1, w.Hq, w.Hkv),
-                                     amax_in=amax_t[b])
+                                     amax_in=amax_t[b], smooth_q=w.smooth_q,
+                                     qmean_in=qmeans[b] if w.smooth_q else None)
         g = got.reshape(-1, w.D) if rows is None else got[rows[:, 0], rows[:, 1]]
-        m = oracle_mod.metrics(g, em.reshape(-1, w.D))
+        e = em.reshape(-1, w.D)
+        m = oracle_mod.metrics(g, e)
         vmax = float(np.abs(vs).max())
-        assert m["max_abs"] <= MAX_ABS_FRAC * vmax, (b, m, vmax)
+        tol = MAX_ABS_FRAC * vmax
         assert m["cos"] >= MIN_COS, (b, m)
+        _check_rows_over_bar(oracle_mod, w, qs, ks, vs, g, e, rows, tol, b)
         worst = m if worst is None or m["cos"] < worst["cos"] else worst
     print(f"\n{w.name}: worst sequence vs emulated {worst}")
 
@@ -241,3 +291,23 @@ def test_dense_entry_equals_general_entry(sage):
     b = sage.sageattn(q, k, v, tensor_layout="HND", is_causal=True)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+def test_q_smoothing_reduces_error_on_shifted_queries(sage, oracle_mod):
+    # Queries sharing a large per-head offset: removing it before quantization and adding
+    # mu_q . k back exactly shrinks the error against exact attention.
+    w = W.general("shifted_queries", 4, 2, 128, (512, 384), seed=74, q_bias_sigma=8.0)
+    x = W.make_general_inputs(w, "cuda")
+    seqs = _per_seq(w, x)
+    errs = {}
+    for sq in (False, True):
+        got = _out_per_seq(w, x, _run(sage, w, x, smooth_q=sq))
+        torch.cuda.synchronize()
+        assert sage.device_error() == 0
+        rel = []
+        for (qs, ks, vs), o in zip(seqs, got):
+            ex = oracle_mod.attn_exact(qs, ks, vs, False, w.sm_scale, heads=(1, w.Hq, w.Hkv))
+            rel.append(oracle_mod.metrics(o, ex)["rel_l1"])
+        errs[sq] = max(rel)
+    print(f"\nrelative L1 vs exact attention without / with Q smoothing: {errs}")
+    assert errs[True] < 0.7 * errs[False], errs
