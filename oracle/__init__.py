@@ -65,6 +65,10 @@ def _L():
             "so_attn_emulated": [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, c_long, c_long, c_long,
                                  c_long, c_long, c_long, c_int, c_double, c_long, vp, c_long, vp],
             "so_qk_bias": [vp, vp, vp, c_long, c_long, c_long, c_long, c_long, vp],
+            "so_quant_int8_rows": [vp, c_long, c_long, c_long, c_long, vp, vp, vp],
+            "so_quant_e4m3_channels": [vp, c_long, c_long, c_long, vp, vp],
+            "so_attn_emulated8": [vp, vp, vp, vp, vp, vp, c_long, c_long, c_long, c_long, c_long,
+                                  c_long, c_long, c_int, c_double, c_long, vp, c_long, vp],
             "so_attn_exact": [vp, vp, vp, c_long, c_long, c_long, c_long, c_long, c_long, c_int,
                               c_double, vp, c_long, vp],
             "so_attn_online": [vp, vp, vp, c_long, c_long, c_long, c_int, c_double, c_long,
@@ -409,6 +413,69 @@ def attn_exact_varlen(q, k, v, cu_q, cu_k, causal: bool, sm_scale: float) -> np.
         o = attn_exact(qs, ks, vs, causal, sm_scale, heads=(1, Hq, Hkv))
         full[cu_q[b]:cu_q[b + 1]] = o.transpose(1, 0, 2)
     return full
+
+
+# ------------------------------------------------------------- 8-bit path --
+
+INT8_BLOCK = 128
+
+
+def quant_int8_rows(x, block: int = INT8_BLOCK, mean=None):
+    """x [G, N, D] -> (int8 codes [G, N, D], scales [G, ceil(N/block)]): symmetric INT8 with
+    one scale fp32(absmax / 127) per block of tokens, codes RNE-rounded and clamped to 127."""
+    x = _f32(x)
+    G, N, D = x.shape
+    nb = (N + block - 1) // block
+    m = None if mean is None else _f32(mean).reshape(G, D)
+    codes = np.zeros((G, N, D), np.int8)
+    sc = np.zeros((G, nb), np.float32)
+    _L().so_quant_int8_rows(_p(x), G, N, D, block, _p(m) if m is not None else None, _p(codes), _p(sc))
+    return codes, sc
+
+
+def quant_e4m3_channels(v):
+    """v [G, N, D] -> (E4M3 codes of V^T [G, D, N], scales [G, D] = fp32(absmax_d / 448))."""
+    v = _f32(v)
+    G, N, D = v.shape
+    codes = np.zeros((G, D, N), np.uint8)
+    sc = np.zeros((G, D), np.float32)
+    _L().so_quant_e4m3_channels(_p(v), G, N, D, _p(codes), _p(sc))
+    return codes, sc
+
+
+def quantize8(q, k, v, smooth_k: bool = True, kmean_in=None, heads=None, block: int = INT8_BLOCK) -> dict:
+    """The 8-bit path's quantization: INT8 Q and (smoothed) K per token block, E4M3 V^T
+    per channel. Shapes as quantize_qkv."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    BHq, Nq, D = q.shape
+    BHkv, Nk, _ = k.shape
+    B, Hq, Hkv = heads if heads is not None else (1, BHq, BHkv)
+    km = np.zeros((BHkv, D), np.float32)
+    if smooth_k:
+        km = _f32(kmean_in).reshape(BHkv, D) if kmean_in is not None else kmean(k)
+    r = {"B": B, "Hq": Hq, "Hkv": Hkv, "Nq": Nq, "Nk": Nk, "D": D, "block": block, "k_mean": km}
+    r["q8"], r["q_scale"] = quant_int8_rows(q, block)
+    r["k8"], r["k_scale"] = quant_int8_rows(k, block, km if smooth_k else None)
+    r["vt8"], r["v_scale"] = quant_e4m3_channels(v)
+    return r
+
+
+def attn_emulated8(qz: dict, causal: bool, sm_scale: float, Bk: int = 128, rows=None) -> np.ndarray:
+    """Emulated 8-bit attention on the output of quantize8 -> [n_rows, D] (or [B*Hq, Nq, D])."""
+    B, Hq, Hkv, Nq, Nk, D = (qz[n] for n in ("B", "Hq", "Hkv", "Nq", "Nk", "D"))
+    r = _rows(B * Hq, Nq, rows)
+    out = np.empty((r.shape[0], D), np.float64)
+    arrs = [np.ascontiguousarray(qz[n]) for n in ("q8", "q_scale", "k8", "k_scale", "vt8", "v_scale")]
+    _L().so_attn_emulated8(*[_p(a) for a in arrs], B, Hq, Hkv, Nq, Nk, D, int(qz["block"]),
+                           int(bool(causal)), float(sm_scale), int(Bk), _p(r), r.shape[0], _p(out))
+    return out.reshape(B * Hq, Nq, D) if rows is None else out
+
+
+def attention8(q, k, v, causal: bool, sm_scale: float, Bk: int = 128, rows=None, smooth_k: bool = True,
+               kmean_in=None, heads=None):
+    """Full emulated 8-bit pipeline."""
+    qz = quantize8(q, k, v, smooth_k=smooth_k, kmean_in=kmean_in, heads=heads)
+    return attn_emulated8(qz, causal, sm_scale, Bk=Bk, rows=rows), qz
 
 
 # ----------------------------------------------------------- error metrics --

@@ -404,6 +404,117 @@ void so_attn_emulated(const uint8_t* q_codes, const uint8_t* q_sf, const uint8_t
   }
 }
 
+// ------------------------------------------------------------ 8-bit path ----
+// The 8-bit forward of the method's training exploration ("An Exploration of 8-Bit
+// Training" in the SageAttention3 title; "trainable INT8 attention" in the SageBwd
+// abstract; INT8 for QK^T per the SageAttention review thread, reply to W1). Formats:
+//   Q, K (K smoothed first): symmetric INT8 with one binary32 scale per block of
+//     `block` consecutive tokens of a head: s = fp32(absmax / 127) (0 -> codes 0),
+//     code = clamp(RNE(fp32(x / s)), -127, 127);
+//   V: E4M3 with one binary32 scale per channel over all tokens of a head:
+//     s_d = fp32(absmax_d / 448), code = E4M3(fp32(v / s_d)) (0 scale -> code 0);
+//   P~: per query row and key tile s1 = rowmax(P~) / 448, code = E4M3(fp32(P~ / s1)).
+
+// x [G, N, D] -> codes [G, N, D] int8, scales [G, ceil(N / block)]; mean [G, D] or NULL.
+void so_quant_int8_rows(const float* x, long G, long N, long D, long block, const float* mean,
+                        int8_t* codes, float* scales) {
+  const long nb = (N + block - 1) / block;
+#pragma omp parallel for schedule(static)
+  for (long gb = 0; gb < G * nb; ++gb) {
+    const long g = gb / nb, b = gb % nb;
+    const long n0 = b * block, n1 = std::min(N, n0 + block);
+    auto val = [&](long n, long d) {
+      float v = x[(g * N + n) * D + d];
+      if (mean) v = v - mean[g * D + d];
+      return v;
+    };
+    float a = 0.0f;
+    for (long n = n0; n < n1; ++n)
+      for (long d = 0; d < D; ++d) a = std::max(a, std::fabs(val(n, d)));
+    const float s = a / 127.0f;
+    scales[g * nb + b] = s;
+    for (long n = n0; n < n1; ++n)
+      for (long d = 0; d < D; ++d) {
+        float c = 0.0f;
+        if (s > 0.0f) c = std::nearbyint(val(n, d) / s);  // default rounding: to nearest even
+        c = std::min(127.0f, std::max(-127.0f, c));
+        codes[(g * N + n) * D + d] = static_cast<int8_t>(c);
+      }
+  }
+}
+
+// v [G, N, D] -> vt codes [G, D, N] (E4M3 bytes), scales [G, D].
+void so_quant_e4m3_channels(const float* v, long G, long N, long D, uint8_t* vt_codes, float* scales) {
+#pragma omp parallel for schedule(static)
+  for (long gd = 0; gd < G * D; ++gd) {
+    const long g = gd / D, d = gd % D;
+    float a = 0.0f;
+    for (long n = 0; n < N; ++n) a = std::max(a, std::fabs(v[(g * N + n) * D + d]));
+    const float s = a / 448.0f;
+    scales[gd] = s;
+    for (long n = 0; n < N; ++n)
+      vt_codes[gd * N + n] = s > 0.0f ? e4m3_encode(v[(g * N + n) * D + d] / s) : 0;
+  }
+}
+
+// Emulated 8-bit attention: dequantize exactly in binary64 (q~ = code * s_q[block], and
+// likewise k~; v~ = e4m3(code) * s_v[d]) and walk key tiles of Bk as so_attn_emulated,
+// with P~ quantized as s1 = rowmax / 448 and p^ = e4m3(fp32(P~ / s1)) * s1.
+// q codes [B*Hq, Nq, D], q scales [B*Hq, ceil(Nq/block)]; k likewise with Hkv, Nk;
+// vt codes [B*Hkv, D, Nk], v scales [B*Hkv, D]. rows (bhq, i); out [n_rows, D].
+void so_attn_emulated8(const int8_t* q_codes, const float* q_scales, const int8_t* k_codes,
+                       const float* k_scales, const uint8_t* vt_codes, const float* v_scales,
+                       long B, long Hq, long Hkv, long Nq, long Nk, long D, long block, int causal,
+                       double sm_scale, long Bk, const long* rows, long n_rows, double* out) {
+  (void)B;
+  const long group = Hq / Hkv;
+  const long nbq = (Nq + block - 1) / block, nbk = (Nk + block - 1) / block;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long r = 0; r < n_rows; ++r) {
+    const long bhq = rows[2 * r], i = rows[2 * r + 1];
+    const long kv = (bhq / Hq) * Hkv + (bhq % Hq) / group;
+    std::vector<double> qd(static_cast<size_t>(D)), O(static_cast<size_t>(D), 0.0);
+    std::vector<double> S(static_cast<size_t>(Bk)), P(static_cast<size_t>(Bk));
+    const double sq = q_scales[bhq * nbq + i / block];
+    for (long d = 0; d < D; ++d) qd[d] = q_codes[(bhq * Nq + i) * D + d] * sq;
+    double m = -std::numeric_limits<double>::infinity(), l = 0.0;
+    const long last_key = causal ? std::min(i + (Nk - Nq), Nk - 1) : Nk - 1;
+    for (long j0 = 0; j0 <= last_key; j0 += Bk) {
+      const long j1 = std::min(j0 + Bk, last_key + 1);
+      double tmax = -std::numeric_limits<double>::infinity();
+      for (long j = j0; j < j1; ++j) {
+        const double sk = k_scales[kv * nbk + j / block];
+        double acc = 0.0;
+        for (long d = 0; d < D; ++d) acc += qd[d] * (k_codes[(kv * Nk + j) * D + d] * sk);
+        S[j - j0] = sm_scale * acc;
+        tmax = std::max(tmax, S[j - j0]);
+      }
+      const double m_new = std::max(m, tmax);
+      const double alpha = std::exp(m - m_new);
+      double rowsum = 0.0, rmax = 0.0;
+      for (long j = j0; j < j1; ++j) {
+        P[j - j0] = std::exp(S[j - j0] - m_new);
+        rowsum += P[j - j0];
+        rmax = std::max(rmax, P[j - j0]);
+      }
+      l = l * alpha + rowsum;
+      const double s1 = rmax / 448.0;
+      for (long j = j0; j < j1; ++j) {
+        const float p2 = static_cast<float>(P[j - j0] / s1);
+        P[j - j0] = e4m3_value(e4m3_encode(p2));
+      }
+      for (long d = 0; d < D; ++d) {
+        const double sv = v_scales[kv * D + d];
+        double acc = 0.0;
+        for (long j = j0; j < j1; ++j) acc += P[j - j0] * (e4m3_value(vt_codes[(kv * D + d) * Nk + j]) * sv);
+        O[d] = O[d] * alpha + s1 * acc;
+      }
+      m = m_new;
+    }
+    for (long d = 0; d < D; ++d) out[r * D + d] = l > 0.0 ? O[d] / l : 0.0;
+  }
+}
+
 // --------------------------------------------------- unquantized attention ----
 // Plain two-pass softmax attention in binary64 on the fp32 inputs (the definition):
 //   O_i = sum_j exp(S_ij - max_j S_ij) v_j / sum_j exp(S_ij - max_j S_ij),
