@@ -352,20 +352,22 @@ def time_general(sage, gw, dev, stream, warmup, steps, inputs=None):
     if gw.packed:
         pr = sage.sageattn_varlen_problem(x["q"], x["k"], x["v"], out, x["cu_seqlens_q"],
                                           x["cu_seqlens_k"], max(gw.lens_q), max(gw.lens_k),
-                                          gw.causal, None, True, gw.gscale, gw.smooth_q)
+                                          gw.causal, None, True, gw.gscale, gw.smooth_q, gw.precision)
     else:
         pr = sage.sageattn_problem(x["q"], x["k"], x["v"], out, gw.layout, gw.causal, None, True,
-                                   gw.gscale, gw.smooth_q)
+                                   gw.gscale, gw.smooth_q, gw.precision)
     ws = torch.empty(sage.problem_sizes(pr)["workspace"], dtype=torch.uint8, device=dev)
 
     def run():
         if gw.packed:
             sage.sageattn_varlen(x["q"], x["k"], x["v"], x["cu_seqlens_q"], x["cu_seqlens_k"],
                                  max(gw.lens_q), max(gw.lens_k), is_causal=gw.causal,
-                                 gscale=gw.gscale, out=out, workspace=ws, smooth_q=gw.smooth_q)
+                                 gscale=gw.gscale, out=out, workspace=ws, smooth_q=gw.smooth_q,
+                                 precision=gw.precision)
         else:
             sage.sageattn(x["q"], x["k"], x["v"], tensor_layout=gw.layout, is_causal=gw.causal,
-                          gscale=gw.gscale, out=out, workspace=ws, smooth_q=gw.smooth_q)
+                          gscale=gw.gscale, out=out, workspace=ws, smooth_q=gw.smooth_q,
+                          precision=gw.precision)
 
     for _ in range(max(warmup, 3)):
         run()
@@ -484,6 +486,10 @@ def main():
         qw = workloads.general(f"{wl.name}_smooth_q", wl.H, wl.H, wl.D, (wl.N,) * wl.B, causal=wl.causal,
                                packed=False, seed=wl.seed, smooth_q=True)
         variants[qw.name] = time_general(sage, qw, dev, stream, args.warmup, min(args.steps, 20),
+                                         inputs=(qd, kd, vd))
+        ew = workloads.general(f"{wl.name}_8bit", wl.H, wl.H, wl.D, (wl.N,) * wl.B, causal=wl.causal,
+                               packed=False, seed=wl.seed, precision="8bit")
+        variants[ew.name] = time_general(sage, ew, dev, stream, args.warmup, min(args.steps, 20),
                                          inputs=(qd, kd, vd))
         gw = workloads.LLM_VARLEN_GQA
         variants[gw.name] = time_general(sage, gw, dev, stream, args.warmup, min(args.steps, 20))

@@ -103,6 +103,14 @@ typedef enum {
   SAGE_GSCALE_HEAD = 2    /* plus one FP32 scale per (sequence, head) of each tensor */
 } sage_gscale_t;
 
+typedef enum {
+  SAGE_PRECISION_FP4 = 0,  /* microscaling FP4 Q, K, P~, V (the method; steps 1-6) */
+  SAGE_PRECISION_8BIT = 1  /* the 8-bit path of the method's training exploration: INT8 Q, K
+                              (after K smoothing) with one scale per 128-token tile, E4M3 V
+                              with one scale per channel, E4M3 P~ with s1 = rowmax / 448 per
+                              row and key tile; no second-level scale, no Q smoothing */
+} sage_precision_t;
+
 /*
  * One attention problem. Element (sequence b, head h, token n, channel d) of Q is at
  *   q + (b*q_stride[0] + h*q_stride[1] + (t0 + n)*q_stride[2] + d) elements,
@@ -130,9 +138,14 @@ typedef struct {
   sage_gscale_t gscale;
   int smooth_q;                 /* subtract the per-(sequence, head) channel mean of Q before
                                    quantizing it, and add mu_q . (k - mu_k) back to the scores */
+  sage_precision_t precision;   /* SAGE_PRECISION_FP4 (0) or SAGE_PRECISION_8BIT */
 } sage_fp4_problem_t;
 
-/* The quantized tensors of a problem (layouts above); device pointers, 16-byte aligned. */
+/* The quantized tensors of a problem (layouts above); device pointers, 16-byte aligned.
+ * With SAGE_PRECISION_8BIT the same fields hold: q_fp4 / k_fp4 int8 codes [rows, D] (one
+ * byte per element), q_sf / k_sf one float32 scale per 128-row tile, vt_fp4 E4M3 codes
+ * [key tiles, D, 128] (V transposed per tile, one byte per token), vt_sf float32 channel
+ * scales [B*Hkv, D]; amax, q_mean and qk_bias are unused. */
 typedef struct {
   uint8_t *q_fp4, *q_sf, *k_fp4, *k_sf, *vt_fp4, *vt_sf;
   float* k_mean;                /* required by sage_fp4_quantize */

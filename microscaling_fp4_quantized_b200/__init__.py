@@ -29,6 +29,7 @@ LIB_PATH = os.environ.get("SAGE_FP4_LIB") or os.path.join(_HERE, "libsage_fp4.so
 SAGE_OK, SAGE_ERR_INVALID_ARG, SAGE_ERR_UNSUPPORTED, SAGE_ERR_CUDA, SAGE_ERR_TIMEOUT = range(5)
 SAGE_BF16, SAGE_F16 = 0, 1
 GSCALE = {"none": 0, "tensor": 1, "head": 2}
+PRECISION = {"fp4": 0, "8bit": 1}
 
 EXPORTED = [
     "sage_status_string", "sage_fp4_quantized_sizes", "sage_fp4_quantize_scratch_bytes",
@@ -64,7 +65,8 @@ class _Problem(ctypes.Structure):
                 ("q_stride", ctypes.c_int64 * 3), ("k_stride", ctypes.c_int64 * 3),
                 ("v_stride", ctypes.c_int64 * 3), ("o_stride", ctypes.c_int64 * 3),
                 ("dtype", ctypes.c_int), ("causal", ctypes.c_int), ("sm_scale", ctypes.c_float),
-                ("smooth_k", ctypes.c_int), ("gscale", ctypes.c_int), ("smooth_q", ctypes.c_int)]
+                ("smooth_k", ctypes.c_int), ("gscale", ctypes.c_int), ("smooth_q", ctypes.c_int),
+                ("precision", ctypes.c_int)]
 
 
 _QZ_FIELDS = ("q_fp4", "q_sf", "k_fp4", "k_sf", "vt_fp4", "vt_sf", "k_mean", "amax", "seq", "q_mean",
@@ -339,10 +341,12 @@ def make_problem(*, B: int, Hq: int, Hkv: int, D: int, Nq: int, Nk: int, dtype: 
                  sm_scale: Optional[float] = None, smooth_k: bool = True, gscale: str = "none",
                  cu_seqlens_q: Optional[torch.Tensor] = None,
                  cu_seqlens_k: Optional[torch.Tensor] = None, total_q: int = 0,
-                 total_k: int = 0, smooth_q: bool = False) -> _Problem:
+                 total_k: int = 0, smooth_q: bool = False, precision: str = "fp4") -> _Problem:
     """The C problem descriptor (strides in elements of (sequence, head, token))."""
     if gscale not in GSCALE:
         raise ValueError(f"gscale must be one of {tuple(GSCALE)}")
+    if precision not in PRECISION:
+        raise ValueError(f"precision must be one of {tuple(PRECISION)}")
     pr = _Problem()
     pr.B, pr.Hq, pr.Hkv, pr.D, pr.Nq, pr.Nk = B, Hq, Hkv, D, Nq, Nk
     pr.cu_seqlens_q = cu_seqlens_q.data_ptr() if cu_seqlens_q is not None else None
@@ -359,6 +363,7 @@ def make_problem(*, B: int, Hq: int, Hkv: int, D: int, Nq: int, Nk: int, dtype: 
     pr.smooth_k = int(bool(smooth_k))
     pr.gscale = GSCALE[gscale]
     pr.smooth_q = int(bool(smooth_q))
+    pr.precision = PRECISION[precision]
     return pr
 
 
@@ -416,7 +421,7 @@ def _same_kind(q, k, v):
 
 def sageattn_problem(q, k, v, out, tensor_layout: str = "HND", is_causal: bool = False,
                      sm_scale: Optional[float] = None, smooth_k: bool = True,
-                     gscale: str = "none", smooth_q: bool = False) -> _Problem:
+                     gscale: str = "none", smooth_q: bool = False, precision: str = "fp4") -> _Problem:
     """The problem descriptor :func:`sageattn` passes to the library."""
     _same_kind(q, k, v)
     if tensor_layout == "HND":
@@ -434,29 +439,34 @@ def sageattn_problem(q, k, v, out, tensor_layout: str = "HND", is_causal: bool =
     return make_problem(B=B, Hq=Hq, Hkv=Hkv, D=D, Nq=Nq, Nk=Nk, dtype=q.dtype,
                         q_stride=_strides3(q, dims), k_stride=_strides3(k, dims),
                         v_stride=_strides3(v, dims), o_stride=_strides3(out, dims), causal=is_causal,
-                        sm_scale=sm_scale, smooth_k=smooth_k, gscale=gscale, smooth_q=smooth_q)
+                        sm_scale=sm_scale, smooth_k=smooth_k, gscale=gscale, smooth_q=smooth_q,
+                        precision=precision)
 
 
 def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tensor_layout: str = "HND",
              is_causal: bool = False, sm_scale: Optional[float] = None, smooth_k: bool = True,
              gscale: str = "none", out: Optional[torch.Tensor] = None,
-             workspace: Optional[torch.Tensor] = None, smooth_q: bool = False) -> torch.Tensor:
+             workspace: Optional[torch.Tensor] = None, smooth_q: bool = False,
+             precision: str = "fp4") -> torch.Tensor:
     """FP4 attention on [B, H, N, D] ("HND") or [B, N, H, D] ("NHD") tensors with any
     strides (channels contiguous). k and v may have fewer heads than q (each shared by
     Hq / Hkv query heads) and a different length (the causal mask then aligns the last
     query with the last key). gscale adds a second-level FP32 scale per tensor ("tensor")
     or per (batch, head) ("head"); smooth_q subtracts each head's query mean before
-    quantization and adds its product with the keys back to the scores."""
+    quantization and adds its product with the keys back to the scores. precision="8bit"
+    runs the 8-bit path instead (INT8 Q/K per 128-token tile, E4M3 P~ and V)."""
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype, device=q.device)
-    pr = sageattn_problem(q, k, v, out, tensor_layout, is_causal, sm_scale, smooth_k, gscale, smooth_q)
+    pr = sageattn_problem(q, k, v, out, tensor_layout, is_causal, sm_scale, smooth_k, gscale, smooth_q,
+                          precision)
     return _run(pr, q, k, v, out, workspace)
 
 
 def sageattn_varlen_problem(q, k, v, out, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
                             max_seqlen_k: int, is_causal: bool = False,
                             sm_scale: Optional[float] = None, smooth_k: bool = True,
-                            gscale: str = "none", smooth_q: bool = False) -> _Problem:
+                            gscale: str = "none", smooth_q: bool = False,
+                            precision: str = "fp4") -> _Problem:
     """The problem descriptor :func:`sageattn_varlen` passes to the library."""
     _same_kind(q, k, v)
     if q.dim() != 3 or k.dim() != 3:
@@ -475,7 +485,7 @@ def sageattn_varlen_problem(q, k, v, out, cu_seqlens_q, cu_seqlens_k, max_seqlen
                       o_stride=_strides3(out, dims), causal=is_causal, sm_scale=sm_scale,
                       smooth_k=smooth_k, gscale=gscale, cu_seqlens_q=cu_seqlens_q,
                       cu_seqlens_k=cu_seqlens_k, total_q=total_q, total_k=total_k,
-                      smooth_q=smooth_q)
+                      smooth_q=smooth_q, precision=precision)
 
 
 def sageattn_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.Tensor,
@@ -483,7 +493,8 @@ def sageattn_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
                     is_causal: bool = False, sm_scale: Optional[float] = None,
                     smooth_k: bool = True, gscale: str = "none",
                     out: Optional[torch.Tensor] = None,
-                    workspace: Optional[torch.Tensor] = None, smooth_q: bool = False) -> torch.Tensor:
+                    workspace: Optional[torch.Tensor] = None, smooth_q: bool = False,
+                    precision: str = "fp4") -> torch.Tensor:
     """FP4 attention on packed sequences: q [total_q, Hq, D], k and v [total_k, Hkv, D];
     sequence b holds tokens cu_seqlens_q[b] .. cu_seqlens_q[b+1] (int32 CUDA tensors of
     B+1 offsets; a bad table is reported by device_error(), never by a fault). Each
@@ -491,5 +502,5 @@ def sageattn_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype, device=q.device)
     pr = sageattn_varlen_problem(q, k, v, out, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
-                                 max_seqlen_k, is_causal, sm_scale, smooth_k, gscale, smooth_q)
+                                 max_seqlen_k, is_causal, sm_scale, smooth_k, gscale, smooth_q, precision)
     return _run(pr, q, k, v, out, workspace)

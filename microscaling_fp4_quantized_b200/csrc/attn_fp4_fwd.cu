@@ -34,12 +34,18 @@
 
 #include <cstdint>
 
+#include "attn_common.cuh"
 #include "sage_internal.h"
 #include "sm100_ptx.cuh"
 
 namespace sage {
 
 namespace {
+
+using attn::Ctl;
+using attn::store_out8;
+using attn::tmem_wait_regs;
+using attn::wait_bar;
 
 constexpr int kStages = 3;
 constexpr int kSoftmaxWarps = 8;
@@ -107,40 +113,6 @@ enum : int {
 };
 static_assert(B_COUNT <= 32, "barrier area");
 
-struct Ctl {
-  volatile uint32_t* abort;
-  uint32_t* err;
-  uint64_t timeout_ns;
-};
-
-// Bounded wait: true when the phase with `parity` has completed, false on abort/timeout.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& c) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*c.abort) return false;
-    if (globaltimer_ns() - t0 > c.timeout_ns) {
-      *c.abort = 1u;
-      atomicOr(c.err, kDevErrTimeout);
-      return false;
-    }
-  }
-}
-
-// 32 columns from TMEM, with the wait::ld tied to the registers it produces.
-__device__ __forceinline__ void tmem_wait_regs(uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.wait::ld.sync.aligned;"
-      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
-        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
-        "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
-        "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
-        "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
-      :
-      : "memory");
-}
-
 __device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
   // 32 rows x 16 bytes, 8-row core matrices 128 bytes apart, no swizzle.
   return make_sdesc(saddr, 0, 128, kLayoutNone);
@@ -154,25 +126,6 @@ __device__ __forceinline__ uint64_t qk_desc(uint32_t saddr) {
 
 __device__ __forceinline__ uint64_t row64_desc(uint32_t saddr) {
   return make_sdesc(saddr, 16, 512, kLayoutSw64);
-}
-
-__device__ __forceinline__ void store_out8(void* out, size_t idx, const float* v, int dtype) {
-  uint4 w;
-  uint32_t* ww = reinterpret_cast<uint32_t*>(&w);
-  if (dtype == kDtypeBF16) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-      ww[i] = *reinterpret_cast<uint32_t*>(&h);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
-      ww[i] = *reinterpret_cast<uint32_t*>(&h);
-    }
-  }
-  *reinterpret_cast<uint4*>(static_cast<char*>(out) + idx * 2) = w;
 }
 
 }  // namespace

@@ -264,6 +264,11 @@ __global__ void __launch_bounds__(kThreads) stats_kernel(QuantParams p) {
                            p.ksum + base, gs ? p.kmax + base : nullptr, gs ? p.kmin + base : nullptr,
                            red, redmx, redmn);
   }
+  if (h < p.Hkv && p.bits8 && n0 < si.len_k) {
+    const size_t base = (static_cast<size_t>(b * p.Hkv + h) * p.nsplit + split) * D;
+    chunk_channel_stats<D>(p.v, p.sv, p.dtype, b, h, si.tok_k, n0, min(n0 + kChunk, si.len_k), true,
+                           p.vsum + base, p.vmax + base, p.vmin + base, red, redmx, redmn);
+  }
   if (h < p.Hq && p.smooth_q && n0 < si.len_q) {
     const size_t base = (static_cast<size_t>(b * p.Hq + h) * p.nsplit + split) * D;
     chunk_channel_stats<D>(p.q, p.sq, p.dtype, b, h, si.tok_q, n0, min(n0 + kChunk, si.len_q), gs,
@@ -313,6 +318,16 @@ __global__ void __launch_bounds__(D) finalize_kernel(QuantParams p) {
       mu = static_cast<float>(s / static_cast<double>(si.len_k));
     }
     p.k_mean[static_cast<size_t>(b * p.Hkv + h) * D + d] = mu;
+    if (p.bits8) {
+      // E4M3 scale of V's channel d: fp32(max |v| / 448) over the sequence's tokens.
+      float mx = -INFINITY, mn = INFINITY;
+      for (int g = 0; g < ns; ++g) {
+        mx = fmaxf(mx, p.vmax[base + static_cast<size_t>(g) * D]);
+        mn = fminf(mn, p.vmin[base + static_cast<size_t>(g) * D]);
+      }
+      const float a = si.len_k > 0 ? fmaxf(fabsf(mx), fabsf(mn)) : 0.0f;
+      p.v_scale[static_cast<size_t>(b * p.Hkv + h) * D + d] = __fdiv_rn(a, 448.0f);
+    }
     if (gs) {
       float mx = -INFINITY, mn = INFINITY, av = 0.0f;
       for (int g = 0; g < ns; ++g) {
@@ -541,6 +556,169 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
   uint8_t* sf_out = p.vt_sf + T * 1024;
   for (int i = t; i < 1024 / 16; i += kThreads)
     reinterpret_cast<uint4*>(sf_out)[i] = reinterpret_cast<const uint4*>(sfbuf)[i];
+}
+
+// ------------------------------------------------------------- 8-bit path ----
+// grid (3 * tiles, Hq, B): x = 3 * tile + job. Jobs 0 and 1 turn a 128-row tile of Q or
+// K - mean into symmetric INT8 with one scale s = fp32(absmax / 127) for the tile and
+// codes clamp(RNE(fp32(x / s)), -127, 127); job 2 turns a 128-token tile of V into E4M3
+// codes fp32(v / s_d) with the channel scales of the finalize pass, transposed (tokens
+// contiguous) and stored tile-major [key tiles, D, 128].
+template <int D>
+__global__ void __launch_bounds__(kThreads) quant8_kernel(QuantParams p) {
+  constexpr int CPR = D / 8;
+  constexpr int kVRowBytes = (D + 8) * 2;  // padded V tile row (16-byte multiple)
+  constexpr int kCodeRow = 144;            // padded V^T code staging row (128 used)
+  __shared__ __align__(16) uint8_t smem[128 * kVRowBytes + D * 4];
+  __shared__ float redw[kThreads / 32];
+  static_assert(D * kCodeRow <= 128 * kVRowBytes, "V^T codes reuse the V tile's staging");
+  if (seq_table_bad(p.seq)) return;
+  const int t = threadIdx.x;
+  const int job = blockIdx.x % 3, tile = blockIdx.x / 3, h = blockIdx.y, b = blockIdx.z;
+  const int H = job == 0 ? p.Hq : p.Hkv;
+  if (h >= H) return;
+  const SeqInfo si = seq_info(p.seq, b);
+  const int len = job == 0 ? si.len_q : si.len_k;
+  const int ntile = (len + 127) >> 7;
+  if (tile >= ntile) return;
+  const int prow = job == 0 ? si.prow_q : si.prow_k;
+  const int64_t tok0 = static_cast<int64_t>(job == 0 ? si.tok_q : si.tok_k) + tile * 128;
+  const int64_t row0 = static_cast<int64_t>(H) * prow + static_cast<int64_t>(h) * ntile * 128 + tile * 128;
+  const int64_t T = row0 >> 7;
+  const int rows = min(128, len - tile * 128);
+  constexpr int kRowStep = kThreads / CPR, kIter = 128 / kRowStep;
+  const int c = t % CPR, rl0 = t / CPR;
+
+  if (job < 2) {
+    float* mu = reinterpret_cast<float*>(smem);
+    const bool smooth = job == 1 && p.smooth_k;
+    for (int d = t; d < D; d += kThreads)
+      mu[d] = smooth ? p.k_mean[static_cast<size_t>(b * p.Hkv + h) * D + d] : 0.0f;
+    __syncthreads();
+    float m8[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m8[e] = mu[c * 8 + e];
+    const void* src = job == 0 ? p.q : p.k;
+    const Strides& st = job == 0 ? p.sq : p.sk;
+    uint4 raw[kIter];
+#pragma unroll
+    for (int it = 0; it < kIter; ++it) {
+      const int rl = rl0 + it * kRowStep;
+      raw[it] = rl < rows ? ld_nc_16(row_ptr(src, st, b, h, tok0 + rl) + c * 16) : make_uint4(0, 0, 0, 0);
+    }
+    auto values = [&](int it, float (&x)[8]) {
+      unpack8(raw[it], p.dtype, x);
+      if (smooth && rl0 + it * kRowStep < rows) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], m8[e]);
+      }
+    };
+    float a = 0.0f;
+#pragma unroll
+    for (int it = 0; it < kIter; ++it) {
+      float x[8];
+      values(it, x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(x[e]));
+    }
+    a = block_max(a, redw);
+    const float s = __fdiv_rn(a, 127.0f);
+    if (t == 0) reinterpret_cast<float*>(job == 0 ? p.q_sf : p.k_sf)[T] = s;
+    uint8_t* dst = (job == 0 ? p.q_fp4 : p.k_fp4) + row0 * D;
+#pragma unroll
+    for (int it = 0; it < kIter; ++it) {
+      float x[8];
+      values(it, x);
+      uint32_t w[2] = {0u, 0u};
+      if (s > 0.0f) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float r = fminf(127.0f, fmaxf(-127.0f, rintf(__fdiv_rn(x[e], s))));
+          w[e >> 2] |= (static_cast<uint32_t>(static_cast<int>(r)) & 0xFFu) << (8 * (e & 3));
+        }
+      }
+      *reinterpret_cast<uint2*>(dst + static_cast<size_t>(rl0 + it * kRowStep) * D + c * 8) = make_uint2(w[0], w[1]);
+    }
+    return;
+  }
+
+  // ---- V^T: E4M3 with one scale per channel ----
+  uint8_t* vtile = smem;                                         // 128 x kVRowBytes
+  float* sv = reinterpret_cast<float*>(smem + 128 * kVRowBytes); // D channel scales
+  for (int d = t; d < D; d += kThreads) sv[d] = p.v_scale[static_cast<size_t>(b * p.Hkv + h) * D + d];
+  {
+    uint4 raw[kIter];
+#pragma unroll
+    for (int it = 0; it < kIter; ++it) {
+      const int rl = rl0 + it * kRowStep;
+      raw[it] = rl < rows ? ld_nc_16(row_ptr(p.v, p.sv, b, h, tok0 + rl) + c * 16) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int it = 0; it < kIter; ++it)
+      *reinterpret_cast<uint4*>(vtile + (rl0 + it * kRowStep) * kVRowBytes + c * 16) = raw[it];
+  }
+  __syncthreads();
+  constexpr int kItems = D * 8 / kThreads;  // (channel, 16-token block) pairs per thread
+  uint4 codes[kItems];
+#pragma unroll
+  for (int k = 0; k < kItems; ++k) {
+    const int item = t + k * kThreads;
+    const int d = item % D, tb = item / D;
+    const float s = sv[d];
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (s > 0.0f) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint16_t hv = *reinterpret_cast<const uint16_t*>(vtile + (tb * 16 + i) * kVRowBytes + d * 2);
+        const float x = (p.dtype == kDtypeBF16) ? __uint_as_float(static_cast<uint32_t>(hv) << 16)
+                                                : __half2float(__ushort_as_half(hv));
+        w[i >> 2] |= f32_to_e4m3(__fdiv_rn(x, s)) << (8 * (i & 3));
+      }
+    }
+    codes[k] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  __syncthreads();  // the tile is read; its storage now stages the codes
+  uint8_t* cbuf = smem;
+#pragma unroll
+  for (int k = 0; k < kItems; ++k) {
+    const int item = t + k * kThreads;
+    *reinterpret_cast<uint4*>(cbuf + (item % D) * kCodeRow + (item / D) * 16) = codes[k];
+  }
+  __syncthreads();
+  uint8_t* vt = p.vt_fp4 + T * (D * 128);
+  for (int gi = t; gi < D * 8; gi += kThreads) {
+    const int d = gi / 8, k = gi % 8;
+    *reinterpret_cast<uint4*>(vt + d * 128 + k * 16) = *reinterpret_cast<const uint4*>(cbuf + d * kCodeRow + k * 16);
+  }
+}
+
+cudaError_t launch_quantize8(const QuantParams& p, const QuantLaunch& l, cudaStream_t stream) {
+  if (p.B == 0 || p.Hq == 0) return cudaSuccess;
+  if (p.seq.cu_q != nullptr) {
+    seq_plan_kernel<<<1, 1024, 0, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (p.nsplit > 0) {
+    dim3 g1(p.nsplit, p.Hq, p.B);
+    if (p.D == 64) stats_kernel<64><<<g1, kThreads, 0, stream>>>(p);
+    else stats_kernel<128><<<g1, kThreads, 0, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  {
+    dim3 g2(p.Hq, p.B);
+    if (p.D == 64) finalize_kernel<64><<<g2, 64, 0, stream>>>(p);
+    else finalize_kernel<128><<<g2, 128, 0, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const int tiles = l.tiles_q > l.tiles_k ? l.tiles_q : l.tiles_k;
+  if (tiles == 0) return cudaSuccess;
+  dim3 g3(3 * tiles, p.Hq, p.B);
+  if (p.D == 64) quant8_kernel<64><<<g3, kThreads, 0, stream>>>(p);
+  else quant8_kernel<128><<<g3, kThreads, 0, stream>>>(p);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_quantize(const QuantParams& p, const QuantLaunch& l, cudaStream_t stream) {

@@ -92,7 +92,7 @@ size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 // A checked problem with everything derived from it.
 struct Prob {
   sage_fp4_problem_t u;  // the caller's description (sm_scale resolved)
-  bool packed, empty, gs, sq;
+  bool packed, empty, gs, sq, b8;
   int64_t rows_q, rows_k;  // padded token rows per head (packed: an upper bound)
   int tiles_q, tiles_k, nsplit;
 };
@@ -118,6 +118,9 @@ sage_status_t check_problem(const sage_fp4_problem_t* in, Prob* p) {
   }
   p->gs = u.gscale != SAGE_GSCALE_NONE;
   p->sq = u.smooth_q != 0;
+  if (u.precision != SAGE_PRECISION_FP4 && u.precision != SAGE_PRECISION_8BIT) return SAGE_ERR_INVALID_ARG;
+  p->b8 = u.precision == SAGE_PRECISION_8BIT;
+  if (p->b8 && (p->gs || p->sq)) return SAGE_ERR_UNSUPPORTED;
   const int64_t* strides[4] = {p->u.q_stride, p->u.k_stride, p->u.v_stride, p->u.o_stride};
   for (const int64_t* s : strides)
     for (int i = 0; i < 3; ++i)
@@ -153,6 +156,22 @@ sage_fp4_problem_sizes_t sizes_of(const Prob& p) {
   std::memset(&z, 0, sizeof(z));
   if (p.empty) return z;
   const int64_t D = p.u.D, B = p.u.B, Hq = p.u.Hq, Hkv = p.u.Hkv;
+  if (p.b8) {
+    const int64_t ns = p.nsplit;
+    z.q_fp4 = static_cast<size_t>(Hq * p.rows_q * D);
+    z.q_sf = static_cast<size_t>(Hq * p.rows_q / 128 * 4);
+    z.k_fp4 = static_cast<size_t>(Hkv * p.rows_k * D);
+    z.k_sf = static_cast<size_t>(Hkv * p.rows_k / 128 * 4);
+    z.vt_fp4 = static_cast<size_t>(Hkv * p.rows_k * D);
+    z.vt_sf = static_cast<size_t>(B * Hkv * D * 4);
+    z.k_mean = static_cast<size_t>(B * Hkv * D * 4);
+    z.amax = 0;
+    z.seq = p.packed ? static_cast<size_t>((2 * (B + 1) + 4) * 4) : 0;
+    z.scratch = up256(static_cast<size_t>(B * Hkv * ns * D * 8)) * 2 + 2 * up256(static_cast<size_t>(B * Hkv * ns * D * 4));
+    z.workspace = up256(z.q_fp4) + up256(z.q_sf) + up256(z.k_fp4) + up256(z.k_sf) + up256(z.vt_fp4) +
+                  up256(z.vt_sf) + up256(z.k_mean) + up256(z.seq) + z.scratch;
+    return z;
+  }
   z.q_fp4 = static_cast<size_t>(Hq * p.rows_q * D / 2);
   z.q_sf = static_cast<size_t>(Hq * p.rows_q * D / 16);
   z.k_fp4 = static_cast<size_t>(Hkv * p.rows_k * D / 2);
@@ -192,7 +211,7 @@ void carve(const Prob& p, void* base, sage_fp4_quantized_t* qz, void** scratch) 
   qz->vt_fp4 = take(z.vt_fp4);
   qz->vt_sf = take(z.vt_sf);
   qz->k_mean = reinterpret_cast<float*>(take(z.k_mean));
-  qz->amax = reinterpret_cast<float*>(take(z.amax));
+  qz->amax = z.amax ? reinterpret_cast<float*>(take(z.amax)) : nullptr;
   qz->seq = p.packed ? reinterpret_cast<int32_t*>(take(z.seq)) : nullptr;
   qz->q_mean = p.sq ? reinterpret_cast<float*>(take(z.q_mean)) : nullptr;
   qz->qk_bias = p.sq ? take(z.qk_bias) : nullptr;
@@ -225,6 +244,7 @@ sage_status_t check_bundle(const Prob& p, const sage_fp4_quantized_t* qz, bool n
     if (ptr == nullptr || !aligned16(ptr)) return SAGE_ERR_INVALID_ARG;
   if (need_kmean && (qz->k_mean == nullptr || !aligned16(qz->k_mean))) return SAGE_ERR_INVALID_ARG;
   if (p.gs && (qz->amax == nullptr || !aligned16(qz->amax))) return SAGE_ERR_INVALID_ARG;
+  if (p.b8 && need_kmean && (qz->k_mean == nullptr || !aligned16(qz->k_mean))) return SAGE_ERR_INVALID_ARG;
   if (p.packed && (qz->seq == nullptr || !aligned16(qz->seq))) return SAGE_ERR_INVALID_ARG;
   if (p.sq && (qz->qk_bias == nullptr || !aligned16(qz->qk_bias))) return SAGE_ERR_INVALID_ARG;
   if (p.sq && need_kmean && (qz->q_mean == nullptr || !aligned16(qz->q_mean))) return SAGE_ERR_INVALID_ARG;
@@ -251,6 +271,7 @@ sage_status_t run_quantize(const Prob& p, const void* q, const void* k, const vo
   k_.seq = seq_map(p, qz);
   k_.smooth_k = p.u.smooth_k ? 1 : 0;
   k_.smooth_q = p.sq ? 1 : 0;
+  k_.bits8 = p.b8 ? 1 : 0;
   k_.q_mean = p.sq ? qz.q_mean : nullptr;
   k_.qk_bias = p.sq ? qz.qk_bias : nullptr;
   k_.gscale = p.u.gscale;
@@ -267,7 +288,16 @@ sage_status_t run_quantize(const Prob& p, const void* q, const void* k, const vo
   const int64_t B = p.u.B, Hq = p.u.Hq, Hkv = p.u.Hkv, ns = p.nsplit, D = p.u.D;
   uint8_t* s = static_cast<uint8_t*>(scratch);
   auto take = [&](size_t n) { uint8_t* r = s; s += up256(n); return r; };
-  if (p.u.smooth_k || p.gs || p.sq) k_.ksum = reinterpret_cast<double*>(take(static_cast<size_t>(B * Hkv * ns * D * 8)));
+  if (p.b8) {
+    // 8-bit path: K sums, then V channel sums / maxima / minima (the sums are not used).
+    k_.ksum = reinterpret_cast<double*>(take(static_cast<size_t>(B * Hkv * ns * D * 8)));
+    k_.vsum = reinterpret_cast<double*>(take(static_cast<size_t>(B * Hkv * ns * D * 8)));
+    k_.vmax = reinterpret_cast<float*>(take(static_cast<size_t>(B * Hkv * ns * D * 4)));
+    k_.vmin = reinterpret_cast<float*>(take(static_cast<size_t>(B * Hkv * ns * D * 4)));
+    k_.v_scale = reinterpret_cast<float*>(qz.vt_sf);
+  } else if (p.u.smooth_k || p.gs || p.sq) {
+    k_.ksum = reinterpret_cast<double*>(take(static_cast<size_t>(B * Hkv * ns * D * 8)));
+  }
   if (p.gs) {
     k_.kmax = reinterpret_cast<float*>(take(static_cast<size_t>(B * Hkv * ns * D * 4)));
     k_.kmin = reinterpret_cast<float*>(take(static_cast<size_t>(B * Hkv * ns * D * 4)));
@@ -287,7 +317,19 @@ sage_status_t run_quantize(const Prob& p, const void* q, const void* k, const vo
     k_.bad_out = reinterpret_cast<uint32_t*>(qz.seq + 2 * (p.u.B + 1));
   }
   k_.err = err;
+  if (p.b8) return cuda_status(sage::launch_quantize8(k_, sage::QuantLaunch{p.tiles_q, p.tiles_k}, stream));
   return cuda_status(sage::launch_quantize(k_, sage::QuantLaunch{p.tiles_q, p.tiles_k}, stream));
+}
+
+sage_status_t build_maps8(const Prob& p, const uint8_t* q8, const uint8_t* k8, const uint8_t* vt8,
+                          sage::TensorMaps* m) {
+  const uint64_t D = static_cast<uint64_t>(p.u.D);
+  const CUtensorMapSwizzle swqk = D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  sage_status_t st;
+  if ((st = make_map(&m->q, q8, D, p.u.Hq * p.rows_q, static_cast<uint32_t>(D), 128, swqk)) != SAGE_OK) return st;
+  if ((st = make_map(&m->k, k8, D, p.u.Hkv * p.rows_k, static_cast<uint32_t>(D), 128, swqk)) != SAGE_OK) return st;
+  return make_map(&m->v, vt8, 128, p.u.Hkv * p.rows_k / 128 * D, 128, static_cast<uint32_t>(D),
+                  CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 sage_status_t build_maps(const Prob& p, const uint8_t* q_fp4, const uint8_t* k_fp4, const uint8_t* vt_fp4,
@@ -320,7 +362,11 @@ sage_status_t base_params(int D, float sm_scale, int causal, sage::AttnParams* a
 
 sage_status_t run_attention(const Prob& p, const sage_fp4_quantized_t& qz, void* out, cudaStream_t stream) {
   sage::TensorMaps m;
-  if (sage_status_t st = build_maps(p, qz.q_fp4, qz.k_fp4, qz.vt_fp4, &m); st != SAGE_OK) return st;
+  if (p.b8) {
+    if (sage_status_t st = build_maps8(p, qz.q_fp4, qz.k_fp4, qz.vt_fp4, &m); st != SAGE_OK) return st;
+  } else if (sage_status_t st = build_maps(p, qz.q_fp4, qz.k_fp4, qz.vt_fp4, &m); st != SAGE_OK) {
+    return st;
+  }
   sage::AttnParams a;
   if (sage_status_t st = base_params(p.u.D, p.u.sm_scale, p.u.causal, &a); st != SAGE_OK) return st;
   a.q_sf = qz.q_sf;
@@ -336,6 +382,13 @@ sage_status_t run_attention(const Prob& p, const sage_fp4_quantized_t& qz, void*
   a.seq = seq_map(p, qz);
   a.amax = p.gs ? qz.amax : nullptr;
   a.qk_bias = p.sq ? qz.qk_bias : nullptr;
+  if (p.b8) {
+    a.q_scale8 = reinterpret_cast<const float*>(qz.q_sf);
+    a.k_scale8 = reinterpret_cast<const float*>(qz.k_sf);
+    a.v_scale8 = reinterpret_cast<const float*>(qz.vt_sf);
+    a.amax = nullptr;
+    return cuda_status(sage::launch_attention8(m, a, p.tiles_q, stream));
+  }
   a.gscale = p.u.gscale;
   a.amax_stride = p.u.B * p.u.Hq;
   return cuda_status(sage::launch_attention(m, a, p.tiles_q, stream));

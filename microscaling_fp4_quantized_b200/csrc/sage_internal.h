@@ -90,6 +90,7 @@ struct QuantParams {
   SeqMap seq;
   int smooth_k;
   int smooth_q;      // subtract the per-(sequence, head) query mean; emit the per-key bias
+  int bits8;         // the 8-bit path: INT8 Q/K per 128-token tile, E4M3 V^T per channel
   int gscale;
   int nsplit;        // 512-token chunks of the longest sequence
   int amax_stride;   // B * Hq: distance between the Q, K and V maxima
@@ -112,6 +113,12 @@ struct QuantParams {
   float* qmin;       // [B * Hq, nsplit, D]
   float* qamax;      // [B * Hq, nsplit]
   float* vamax;      // [B * Hkv, nsplit]
+  // 8-bit path: q_fp4 / k_fp4 hold int8 codes [rows, D], q_sf / k_sf one float scale per
+  // 128-row tile, vt_fp4 E4M3 codes [key tiles, D, 128], v_scale the channel scales.
+  float* v_scale;    // [B * Hkv, D]
+  double* vsum;      // [B * Hkv, nsplit, D]  (channel statistics of V, 8-bit path)
+  float* vmax;       // [B * Hkv, nsplit, D]
+  float* vmin;       // [B * Hkv, nsplit, D]
   // Packed problems: the plan kernel's inputs and outputs.
   int total_q, total_k;
   int32_t* pad_q_out;
@@ -132,6 +139,9 @@ struct AttnParams {
   SeqMap seq;
   const float* amax;    // second-level maxima, or nullptr
   const uint8_t* qk_bias; // Q-smoothing bias operand per (query head, padded key row), or nullptr
+  const float* q_scale8;  // 8-bit path: scale per 128-row Q tile
+  const float* k_scale8;  // 8-bit path: scale per 128-row K tile
+  const float* v_scale8;  // 8-bit path: [B * Hkv, D] channel scales of V
   int gscale;
   int amax_stride;
   int BH, Np;           // dense S = Q^ K^^T (scores kernel only)
@@ -154,7 +164,9 @@ struct QuantLaunch {
 };
 
 cudaError_t launch_quantize(const QuantParams& p, const QuantLaunch& l, cudaStream_t stream);
+cudaError_t launch_quantize8(const QuantParams& p, const QuantLaunch& l, cudaStream_t stream);
 cudaError_t launch_attention(const TensorMaps& maps, const AttnParams& p, int tiles_q, cudaStream_t stream);
 cudaError_t launch_qk_scores(const TensorMaps& maps, const AttnParams& p, cudaStream_t stream);
+cudaError_t launch_attention8(const TensorMaps& maps, const AttnParams& p, int tiles_q, cudaStream_t stream);
 
 }  // namespace sage

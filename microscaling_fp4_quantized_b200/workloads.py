@@ -148,6 +148,7 @@ class GeneralWorkload:
     gscale: str = "none"
     smooth_q: bool = False
     q_bias_sigma: float = 0.0
+    precision: str = "fp4"
 
     @property
     def B(self) -> int:
@@ -170,7 +171,8 @@ class GeneralWorkload:
                 "total_q": sum(self.lens_q), "total_k": sum(self.lens_k), "causal": self.causal,
                 "packed": self.packed, "layout": self.layout,
                 "dtype": str(self.dtype).replace("torch.", ""), "seed": self.seed,
-                "gscale": self.gscale, "smooth_q": self.smooth_q, "q_bias_sigma": self.q_bias_sigma}
+                "gscale": self.gscale, "smooth_q": self.smooth_q, "q_bias_sigma": self.q_bias_sigma,
+                "precision": self.precision}
 
 
 def general(name: str, Hq: int, Hkv: int, D: int, lens_q, lens_k=None, causal: bool = False,

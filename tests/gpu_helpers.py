@@ -158,3 +158,43 @@ def sample_rows(N: int, count: int, seed: int) -> np.ndarray:
     base = [0, N - 1, min(N - 1, 127), min(N - 1, 128)]
     extra = rng.choice(N, size=min(N, count), replace=False)
     return np.unique(np.concatenate([base, extra]))
+
+
+def canonical8(qz: dict, lens_q, lens_k, Hq: int, Hkv: int, D: int) -> list:
+    """Per sequence, the GPU's 8-bit quantized tensors in the oracle's layouts: q8 [Hq, Lq, D]
+    int8, q_scale [Hq, ceil(Lq/128)], k8 / k_scale likewise with Hkv, vt8 [Hkv, D, Lk]
+    (E4M3 bytes), v_scale [Hkv, D], k_mean [Hkv, D]; plus pads_zero."""
+    g = {k: qz[k].cpu().numpy() for k in ("q_fp4", "q_sf", "k_fp4", "k_sf", "vt_fp4", "vt_sf")}
+    q_scale, k_scale, v_scale = (g[n].view(np.float32) for n in ("q_sf", "k_sf", "vt_sf"))
+    kmean = qz["k_mean"].cpu().numpy()
+    pq, pk = padded_offsets(lens_q), padded_offsets(lens_k)
+    res = []
+    for b, (Lq, Lk) in enumerate(zip(lens_q, lens_k)):
+        Pq, Pk = (Lq + 127) // 128 * 128, (Lk + 127) // 128 * 128
+        o = {"pads_zero": True}
+        q8, qs = [], []
+        for h in range(Hq):
+            r0 = Hq * pq[b] + h * Pq
+            blk = g["q_fp4"][r0 * D:(r0 + Pq) * D].reshape(Pq, D)
+            q8.append(blk[:Lq].view(np.int8))
+            qs.append(q_scale[r0 // 128:(r0 + Pq) // 128])
+            o["pads_zero"] &= not blk[Lq:].any()
+        k8, ks, vt, vs = [], [], [], []
+        for h in range(Hkv):
+            r0 = Hkv * pk[b] + h * Pk
+            blk = g["k_fp4"][r0 * D:(r0 + Pk) * D].reshape(Pk, D)
+            k8.append(blk[:Lk].view(np.int8))
+            ks.append(k_scale[r0 // 128:(r0 + Pk) // 128])
+            o["pads_zero"] &= not blk[Lk:].any()
+            t0 = r0 // 128
+            t = g["vt_fp4"][t0 * D * 128:(t0 + Pk // 128) * D * 128].reshape(Pk // 128, D, 128)
+            t = t.transpose(1, 0, 2).reshape(D, Pk)
+            vt.append(t[:, :Lk])
+            o["pads_zero"] &= not t[:, Lk:].any()
+            vs.append(v_scale[(b * Hkv + h) * D:(b * Hkv + h + 1) * D])
+        o["q8"], o["q_scale"] = np.stack(q8), np.stack(qs)
+        o["k8"], o["k_scale"] = np.stack(k8), np.stack(ks)
+        o["vt8"], o["v_scale"] = np.stack(vt), np.stack(vs)
+        o["k_mean"] = kmean[b * Hkv * D:(b + 1) * Hkv * D].reshape(Hkv, D)
+        res.append(o)
+    return res

@@ -113,3 +113,16 @@ def test_packed_problem_needs_both_tables(L):
     with pytest.raises(sage.SageError) as e:
         sage.problem_sizes(_dense_pr(sage, cu_seqlens_q=cu, total_q=10, total_k=10))
     assert e.value.status == sage.SAGE_ERR_INVALID_ARG
+
+
+def test_8bit_problem_sizes_and_refusals(L):
+    import microscaling_fp4_quantized_b200 as sage
+    z = sage.problem_sizes(_dense_pr(sage, precision="8bit"))
+    # one byte per element, one float per 128-row tile, float channel scales for V
+    assert z["q_fp4"] == 8 * 2 * 384 * 128 and z["q_sf"] == 8 * 2 * 3 * 4
+    assert z["k_fp4"] == 2 * 2 * 512 * 128 and z["vt_fp4"] == z["k_fp4"] and z["k_sf"] == 2 * 2 * 4 * 4
+    assert z["vt_sf"] == 2 * 2 * 128 * 4 and z["amax"] == 0 and z["qk_bias"] == 0
+    for bad in (dict(gscale="tensor"), dict(smooth_q=True)):
+        with pytest.raises(sage.SageError) as e:
+            sage.problem_sizes(_dense_pr(sage, precision="8bit", **bad))
+        assert e.value.status == sage.SAGE_ERR_UNSUPPORTED
