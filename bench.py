@@ -101,12 +101,13 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
 
 
-def _attn_traffic(wl):
+def _attn_traffic(wl, b8=False):
     """DRAM bytes per attention launch from the committed ncu capture, or None when the
     kernel source has changed since the capture (or no capture exists)."""
     import hashlib
+    name = "attn8_fwd_kernel_traffic.json" if b8 else "attn_fp4_fwd_kernel_traffic.json"
     try:
-        with open(os.path.join(ROOT, "profiles", "attn_fp4_fwd_kernel_traffic.json")) as f:
+        with open(os.path.join(ROOT, "profiles", name)) as f:
             rec = json.load(f)
         with open(os.path.join(ROOT, rec["source"]), "rb") as f:
             sha = hashlib.sha256(f.read()).hexdigest()
@@ -268,7 +269,7 @@ def run_sweep(args):
     return 0
 
 
-def time_e2e(sage, wl, q, k, v, dev, stream, steps, dist, world):
+def time_e2e(sage, wl, q, k, v, dev, stream, steps, dist, world, precision="fp4"):
     """End to end through the public API: every step copies its inputs from pinned host
     memory, runs sage.attn, and copies the output back to pinned host memory.
     Pipelined (the headline): a copy-in stream, the compute stream and a copy-out stream
@@ -279,7 +280,13 @@ def time_e2e(sage, wl, q, k, v, dev, stream, steps, dist, world):
     hout = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(2)]
     din = [tuple(torch.empty(q.shape, dtype=q.dtype, device=dev) for _ in range(3)) for _ in range(2)]
     dout = [torch.empty(q.shape, dtype=q.dtype, device=dev) for _ in range(2)]
-    ws = torch.empty(max(sage.workspace_bytes(wl.B, wl.H, wl.N, wl.D), 256), dtype=torch.uint8, device=dev)
+    ws_bytes = sage.problem_sizes(sage.sageattn_problem(din[0][0], din[0][1], din[0][2], dout[0], "HND", wl.causal,
+                                                        wl.sm_scale, precision=precision))["workspace"]
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+
+    def forward(a, b, c, o):
+        return sage.sageattn(a, b, c, is_causal=wl.causal, sm_scale=wl.sm_scale, out=o, workspace=ws,
+                             precision=precision)
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
     def pipelined(n):
@@ -300,7 +307,7 @@ def time_e2e(sage, wl, q, k, v, dev, stream, steps, dist, world):
             stream.wait_event(ev_in[i])
             if i >= 2:
                 stream.wait_event(ev_out[i - 2])           # output buffer b read back
-            sage.attn(*din[b], causal=wl.causal, sm_scale=wl.sm_scale, out=dout[b], workspace=ws)
+            forward(*din[b], dout[b])
             ev_c[i].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_c[i])
@@ -316,7 +323,7 @@ def time_e2e(sage, wl, q, k, v, dev, stream, steps, dist, world):
         t0.record(stream)
         for _ in range(n):
             a, b, c = (h.to(dev, non_blocking=True) for h in hin[0])
-            o = sage.attn(a, b, c, causal=wl.causal, sm_scale=wl.sm_scale)
+            o = forward(a, b, c, torch.empty_like(a))
             hout[0].copy_(o, non_blocking=True)
         t1.record(stream)
         torch.cuda.synchronize(dev)
@@ -399,6 +406,8 @@ def main():
     ap.add_argument("--variants", action="store_true",
                     help="also time the general-problem paths (second-level scales, packed "
                          "grouped-query batch) and report them under 'variants'")
+    ap.add_argument("--precision", default="fp4", choices=["fp4", "8bit"],
+                    help="the method's FP4 path (default) or its 8-bit path")
     ap.add_argument("--sweep", action="store_true",
                     help="measure every named configuration (one JSON line each) instead of "
                          "the single bench line")
@@ -425,14 +434,15 @@ def main():
     q, k, v = workloads.make_inputs(wl)          # CPU, seeded
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     out = torch.empty_like(qd)
-    plan = sage.Plan(wl.B, wl.H, wl.N, wl.D, wl.dtype, dev)
+    plan = sage.ProblemPlan(sage.sageattn_problem(qd, kd, vd, out, "HND", wl.causal, wl.sm_scale,
+                                                  precision=args.precision), dev)
     stream = torch.cuda.current_stream(dev)
 
     def step(ev_mid=None, ev_end=None):
         plan.quantize(qd, kd, vd)
         if ev_mid is not None:
             ev_mid.record(stream)
-        plan.attention(out, causal=wl.causal, sm_scale=wl.sm_scale)
+        plan.attention(out)
         if ev_end is not None:
             ev_end.record(stream)
 
@@ -473,7 +483,7 @@ def main():
     # --- end to end through the public API: pinned host inputs -> result on the host ---
     e2e = None
     if not args.no_e2e:
-        e2e = time_e2e(sage, wl, q, k, v, dev, stream, max(3, args.steps), dist, world)
+        e2e = time_e2e(sage, wl, q, k, v, dev, stream, max(3, args.steps), dist, world, args.precision)
 
     variants = None
     if args.variants:
@@ -506,12 +516,18 @@ def main():
     fp4_peak = FP4_PER_BF16 * sustained
     attn_avg_ms = statistics.mean(attn_ms)
     achieved = wl.ops / (attn_avg_ms * 1e-3) / 1e12
-    traffic, traffic_src = _attn_traffic(wl)
+    b8 = args.precision == "8bit"
+    traffic, traffic_src = _attn_traffic(wl, b8)
+    if b8:
+        # FP8 / INT8 tensor peak: measured bf16 x 2 (nominal 8-bit : BF16 = 4.5 : 2.25)
+        fp4_peak = 2.0 * sustained
     roofline = {
-        "kernel": "attn_fp4_fwd_kernel", "bound": "tensor", "achieved": achieved, "peak": fp4_peak,
+        "kernel": "attn8_fwd_kernel" if b8 else "attn_fp4_fwd_kernel", "bound": "tensor", "achieved": achieved,
+        "peak": fp4_peak,
         "unit": "TFLOP/s", "frac": achieved / fp4_peak, "traffic": traffic, "traffic_source": traffic_src,
-        "peak_basis": f"{basis} bf16 sustained {sustained} TFLOP/s x {FP4_PER_BF16:g} (nominal FP4:BF16)",
-        "frac_of_nominal_9pflops": achieved / FP4_NOMINAL_TFLOPS,
+        "peak_basis": (f"{basis} bf16 sustained {sustained} TFLOP/s x 2 (nominal 8-bit:BF16)" if b8 else
+                       f"{basis} bf16 sustained {sustained} TFLOP/s x {FP4_PER_BF16:g} (nominal FP4:BF16)"),
+        "frac_of_nominal": achieved / (FP4_NOMINAL_TFLOPS / 2 if b8 else FP4_NOMINAL_TFLOPS),
         "attn_ms": attn_avg_ms, "quant_ms": statistics.mean(quant_ms),
     }
     cpu = None
@@ -519,12 +535,13 @@ def main():
         val, _, sample, cores = cpu_oracle_rate(wl, args.cpu_budget_s)
         cpu = {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
     cfg = wl.describe()
+    cfg["precision"] = args.precision
     cfg["l2"] = "inputs larger than L2 (no flush)"
     cfg["timing"] = "CUDA events on the launching stream, max over ranks"
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "fp4_e2m1", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8_e4m3" if b8 else "fp4_e2m1", "data": "synthetic",
         "config": cfg, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clocks, "device_error_word": err,
         "pct_of_fp4_peak": 100.0 * value / world / fp4_peak,

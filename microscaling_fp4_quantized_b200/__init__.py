@@ -504,3 +504,29 @@ def sageattn_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
     pr = sageattn_varlen_problem(q, k, v, out, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
                                  max_seqlen_k, is_causal, sm_scale, smooth_k, gscale, smooth_q, precision)
     return _run(pr, q, k, v, out, workspace)
+
+
+class ProblemPlan:
+    """Preallocated quantized buffers, scratch and the C problem descriptor for one general
+    problem (see :func:`sageattn_problem` / :func:`sageattn_varlen_problem`): the forward as
+    two C-ABI calls, sage_fp4_quantize and sage_fp4_attn_quantized, with no allocation per
+    call. The tensors passed to quantize() must have the shapes and strides the problem
+    was built from."""
+
+    def __init__(self, problem: _Problem, device="cuda"):
+        self.problem = problem
+        self.device = torch.device(device)
+        z = problem_sizes(problem)
+        self.sizes = z
+        self.buf = {n: torch.empty(max(z[n], 16), dtype=torch.uint8, device=self.device) for n in _QZ_FIELDS}
+        self.scratch = torch.empty(max(z["scratch"], 16), dtype=torch.uint8, device=self.device)
+        self._qz = _Quantized(*[ctypes.c_void_p(self.buf[n].data_ptr()) for n in _QZ_FIELDS])
+
+    def quantize(self, q, k, v) -> None:
+        _check(lib().sage_fp4_quantize(ctypes.byref(self.problem), _ptr(q), _ptr(k), _ptr(v),
+                                       ctypes.byref(self._qz), _ptr(self.scratch), self.sizes["scratch"],
+                                       _stream(self.device)), "sage_fp4_quantize")
+
+    def attention(self, out: torch.Tensor) -> None:
+        _check(lib().sage_fp4_attn_quantized(ctypes.byref(self.problem), ctypes.byref(self._qz), _ptr(out),
+                                             _stream(self.device)), "sage_fp4_attn_quantized")
