@@ -344,8 +344,8 @@ def time_e2e(sage, wl, q, k, v, dev, stream, steps, dist, world, precision="fp4"
             "serial": {"value": job_value(wl.ops, world, ms_s), "ms_per_step": ms_s}}
 
 
-# Kernels per step: K statistics, K mean, quantization, attention.
-LAUNCHES_PER_STEP = 4
+# Kernels per step: K statistics, K mean, Q/K quantization, V^T quantization, attention.
+LAUNCHES_PER_STEP = 5
 
 
 def time_general(sage, gw, dev, stream, warmup, steps, inputs=None):

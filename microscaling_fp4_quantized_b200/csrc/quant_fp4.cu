@@ -4,7 +4,8 @@
 //   stats_kernel     : per 512-token chunk: binary64 column sums of K; with a second-level
 //                      scale also the column maxima / minima of K and the maxima of |Q|, |V|
 //   finalize_kernel  : per (sequence, head): the K mean and the second-level maxima
-//   quant_kernel     : Q, K - mean and V^T -> packed E2M1 codes + UE4M3 scale tiles
+//   quant_kernel     : Q, K - mean (one launch) and V^T (another) -> packed E2M1 codes +
+//                      UE4M3 scale tiles
 //
 // The block rule follows the microscaling FP4 statement of SageAttention3 (arXiv
 // 2505.11594, abstract): per 16 consecutive elements, s = E4M3(absmax / 6) and
@@ -378,18 +379,22 @@ __global__ void __launch_bounds__(D) finalize_kernel(QuantParams p) {
   }
 }
 
-// grid (3 * tiles, Hq, B): x = 3 * tile + job; job 0 quantizes Q rows, 1 K rows
-// (smoothed), 2 V^T. CTAs past a sequence's tiles or heads return at once.
-template <int D>
+// Two launches: VJOB = false, grid (2 * tiles, Hq, B), x = 2 * tile + job, job 0 quantizes
+// Q rows and 1 K rows (smoothed); VJOB = true, grid (key tiles, Hkv, B), V^T. Only the V
+// transpose needs a large shared-memory tile, so the Q/K launch keeps many CTAs per SM.
+// CTAs past a sequence's tiles or heads return at once.
+template <int D, bool VJOB>
 __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
   constexpr int CPR = D / 8;
   constexpr int kVRowBytes = (D + 8) * 2;  // padded V tile row (16-byte multiple)
   constexpr int kCodeRow = 80;             // padded V^T code staging row (64 used)
   constexpr int kSfBytesQK = (D / 64) * 512;
-  __shared__ __align__(16) uint8_t smem[128 * kVRowBytes + D * kCodeRow + 1024 + D * 4];
+  __shared__ __align__(16) uint8_t smem[VJOB ? 128 * kVRowBytes + D * kCodeRow + 1024 : 1024 + D * 4];
   if (seq_table_bad(p.seq)) return;
   const int t = threadIdx.x;
-  const int job = blockIdx.x % 3, tile = blockIdx.x / 3, h = blockIdx.y, b = blockIdx.z;
+  const int job = VJOB ? 2 : static_cast<int>(blockIdx.x % 2);
+  const int tile = VJOB ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x / 2);
+  const int h = blockIdx.y, b = blockIdx.z;
   const int H = job == 0 ? p.Hq : p.Hkv;
   if (h >= H) return;
   const SeqInfo si = seq_info(p.seq, b);
@@ -405,7 +410,7 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
   float g = 1.0f;
   if (gs) g = second_level_scale(p.amax[job * p.amax_stride + (p.gscale == kGscaleHead ? b * H + h : 0)]);
 
-  if (job < 2) {
+  if constexpr (!VJOB) {
     uint8_t* sfbuf = smem;                                  // kSfBytesQK
     float* mu = reinterpret_cast<float*>(smem + 1024);      // D floats
     const bool smooth = (job == 1) ? p.smooth_k != 0 : p.smooth_q != 0;
@@ -500,81 +505,83 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
     uint8_t* sf_out = (job == 0 ? p.q_sf : p.k_sf) + T * kSfBytesQK;
     for (int i = t; i < kSfBytesQK / 16; i += kThreads)
       reinterpret_cast<uint4*>(sf_out)[i] = reinterpret_cast<const uint4*>(sfbuf)[i];
-    return;
-  }
-
-  // ---- V^T: tokens become the contiguous (contraction) dimension ----
-  uint8_t* vtile = smem;                                // 128 x kVRowBytes
-  uint8_t* cbuf = smem + 128 * kVRowBytes;              // D x kCodeRow
-  uint8_t* sfbuf = cbuf + D * kCodeRow;                 // 1024
-  for (int i = t; i < 1024 / 16; i += kThreads) reinterpret_cast<uint4*>(sfbuf)[i] = make_uint4(0, 0, 0, 0);
-  {
-    constexpr int kRowStep = kThreads / CPR, kIter = 128 / kRowStep;
-    const int c = t % CPR, rl0 = t / CPR;
-    uint4 raw[kIter];
-#pragma unroll
-    for (int it = 0; it < kIter; ++it) {
-      const int rl = rl0 + it * kRowStep;
-      raw[it] = rl < rows ? ld_nc_16(row_ptr(p.v, p.sv, b, h, tok0 + rl) + c * 16) : make_uint4(0, 0, 0, 0);
+  } else {
+    // ---- V^T: tokens become the contiguous (contraction) dimension ----
+    uint8_t* vtile = smem;                                // 128 x kVRowBytes
+    uint8_t* cbuf = smem + 128 * kVRowBytes;              // D x kCodeRow
+    uint8_t* sfbuf = cbuf + D * kCodeRow;                 // 1024
+    for (int i = t; i < 1024 / 16; i += kThreads) reinterpret_cast<uint4*>(sfbuf)[i] = make_uint4(0, 0, 0, 0);
+    {
+      constexpr int kRowStep = kThreads / CPR, kIter = 128 / kRowStep;
+      const int c = t % CPR, rl0 = t / CPR;
+      uint4 raw[kIter];
+  #pragma unroll
+      for (int it = 0; it < kIter; ++it) {
+        const int rl = rl0 + it * kRowStep;
+        raw[it] = rl < rows ? ld_nc_16(row_ptr(p.v, p.sv, b, h, tok0 + rl) + c * 16) : make_uint4(0, 0, 0, 0);
+      }
+  #pragma unroll
+      for (int it = 0; it < kIter; ++it)
+        *reinterpret_cast<uint4*>(vtile + (rl0 + it * kRowStep) * kVRowBytes + c * 16) = raw[it];
     }
-#pragma unroll
-    for (int it = 0; it < kIter; ++it)
-      *reinterpret_cast<uint4*>(vtile + (rl0 + it * kRowStep) * kVRowBytes + c * 16) = raw[it];
-  }
-  __syncthreads();
-  for (int item = t; item < D * 8; item += kThreads) {
-    const int d = item % D, tb = item / D;
-    float x[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const uint16_t hv = *reinterpret_cast<const uint16_t*>(vtile + (tb * 16 + i) * kVRowBytes + d * 2);
-      x[i] = (p.dtype == kDtypeBF16) ? __uint_as_float(static_cast<uint32_t>(hv) << 16)
-                                     : __half2float(__ushort_as_half(hv));
-      if (gs) x[i] = __fdiv_rn(x[i], g);
+    __syncthreads();
+    for (int item = t; item < D * 8; item += kThreads) {
+      const int d = item % D, tb = item / D;
+      float x[16];
+  #pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint16_t hv = *reinterpret_cast<const uint16_t*>(vtile + (tb * 16 + i) * kVRowBytes + d * 2);
+        x[i] = (p.dtype == kDtypeBF16) ? __uint_as_float(static_cast<uint32_t>(hv) << 16)
+                                       : __half2float(__ushort_as_half(hv));
+        if (gs) x[i] = __fdiv_rn(x[i], g);
+      }
+      float a = 0.0f;
+  #pragma unroll
+      for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(x[i]));
+      const uint32_t sb = block_scale_byte(a);
+      const float s = e4m3_to_f32(sb);
+      float lo[8], hi[8];
+  #pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        lo[i] = x[i];
+        hi[i] = x[8 + i];
+      }
+      const uint32_t w0 = encode8(lo, s), w1 = encode8(hi, s);
+      *reinterpret_cast<uint2*>(cbuf + d * kCodeRow + tb * 8) = make_uint2(w0, w1);
+      sfbuf[(tb / 4) * 512 + (d % 32) * 16 + (d / 32) * 4 + (tb % 4)] = static_cast<uint8_t>(sb);
     }
-    float a = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(x[i]));
-    const uint32_t sb = block_scale_byte(a);
-    const float s = e4m3_to_f32(sb);
-    float lo[8], hi[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      lo[i] = x[i];
-      hi[i] = x[8 + i];
+    __syncthreads();
+    uint8_t* vt = p.vt_fp4 + T * (D * 64);
+    for (int gi = t; gi < D * 4; gi += kThreads) {
+      const int d = gi / 4, k = gi % 4;
+      *reinterpret_cast<uint4*>(vt + d * 64 + k * 16) = *reinterpret_cast<const uint4*>(cbuf + d * kCodeRow + k * 16);
     }
-    const uint32_t w0 = encode8(lo, s), w1 = encode8(hi, s);
-    *reinterpret_cast<uint2*>(cbuf + d * kCodeRow + tb * 8) = make_uint2(w0, w1);
-    sfbuf[(tb / 4) * 512 + (d % 32) * 16 + (d / 32) * 4 + (tb % 4)] = static_cast<uint8_t>(sb);
+    uint8_t* sf_out = p.vt_sf + T * 1024;
+    for (int i = t; i < 1024 / 16; i += kThreads)
+      reinterpret_cast<uint4*>(sf_out)[i] = reinterpret_cast<const uint4*>(sfbuf)[i];
   }
-  __syncthreads();
-  uint8_t* vt = p.vt_fp4 + T * (D * 64);
-  for (int gi = t; gi < D * 4; gi += kThreads) {
-    const int d = gi / 4, k = gi % 4;
-    *reinterpret_cast<uint4*>(vt + d * 64 + k * 16) = *reinterpret_cast<const uint4*>(cbuf + d * kCodeRow + k * 16);
-  }
-  uint8_t* sf_out = p.vt_sf + T * 1024;
-  for (int i = t; i < 1024 / 16; i += kThreads)
-    reinterpret_cast<uint4*>(sf_out)[i] = reinterpret_cast<const uint4*>(sfbuf)[i];
 }
 
 // ------------------------------------------------------------- 8-bit path ----
-// grid (3 * tiles, Hq, B): x = 3 * tile + job. Jobs 0 and 1 turn a 128-row tile of Q or
-// K - mean into symmetric INT8 with one scale s = fp32(absmax / 127) for the tile and
-// codes clamp(RNE(fp32(x / s)), -127, 127); job 2 turns a 128-token tile of V into E4M3
-// codes fp32(v / s_d) with the channel scales of the finalize pass, transposed (tokens
-// contiguous) and stored tile-major [key tiles, D, 128].
-template <int D>
+// Two launches, split like quant_kernel. VJOB = false, grid (2 * tiles, Hq, B),
+// x = 2 * tile + job: jobs 0 and 1 turn a 128-row tile of Q or K - mean into symmetric
+// INT8 with one scale s = fp32(absmax / 127) for the tile and codes
+// clamp(RNE(fp32(x / s)), -127, 127). VJOB = true, grid (key tiles, Hkv, B): a 128-token
+// tile of V becomes E4M3 codes fp32(v / s_d) with the channel scales of the finalize
+// pass, transposed (tokens contiguous) and stored tile-major [key tiles, D, 128].
+template <int D, bool VJOB>
 __global__ void __launch_bounds__(kThreads) quant8_kernel(QuantParams p) {
   constexpr int CPR = D / 8;
   constexpr int kVRowBytes = (D + 8) * 2;  // padded V tile row (16-byte multiple)
   constexpr int kCodeRow = 144;            // padded V^T code staging row (128 used)
-  __shared__ __align__(16) uint8_t smem[128 * kVRowBytes + D * 4];
+  __shared__ __align__(16) uint8_t smem[VJOB ? 128 * kVRowBytes + D * 4 : D * 4];
   __shared__ float redw[kThreads / 32];
   static_assert(D * kCodeRow <= 128 * kVRowBytes, "V^T codes reuse the V tile's staging");
   if (seq_table_bad(p.seq)) return;
   const int t = threadIdx.x;
-  const int job = blockIdx.x % 3, tile = blockIdx.x / 3, h = blockIdx.y, b = blockIdx.z;
+  const int job = VJOB ? 2 : static_cast<int>(blockIdx.x % 2);
+  const int tile = VJOB ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x / 2);
+  const int h = blockIdx.y, b = blockIdx.z;
   const int H = job == 0 ? p.Hq : p.Hkv;
   if (h >= H) return;
   const SeqInfo si = seq_info(p.seq, b);
@@ -589,7 +596,7 @@ __global__ void __launch_bounds__(kThreads) quant8_kernel(QuantParams p) {
   constexpr int kRowStep = kThreads / CPR, kIter = 128 / kRowStep;
   const int c = t % CPR, rl0 = t / CPR;
 
-  if (job < 2) {
+  if constexpr (!VJOB) {
     float* mu = reinterpret_cast<float*>(smem);
     const bool smooth = job == 1 && p.smooth_k;
     for (int d = t; d < D; d += kThreads)
@@ -639,9 +646,7 @@ __global__ void __launch_bounds__(kThreads) quant8_kernel(QuantParams p) {
       }
       *reinterpret_cast<uint2*>(dst + static_cast<size_t>(rl0 + it * kRowStep) * D + c * 8) = make_uint2(w[0], w[1]);
     }
-    return;
-  }
-
+  } else {
   // ---- V^T: E4M3 with one scale per channel ----
   uint8_t* vtile = smem;                                         // 128 x kVRowBytes
   float* sv = reinterpret_cast<float*>(smem + 128 * kVRowBytes); // D channel scales
@@ -690,6 +695,7 @@ __global__ void __launch_bounds__(kThreads) quant8_kernel(QuantParams p) {
     const int d = gi / 8, k = gi % 8;
     *reinterpret_cast<uint4*>(vt + d * 128 + k * 16) = *reinterpret_cast<const uint4*>(cbuf + d * kCodeRow + k * 16);
   }
+  }
 }
 
 cudaError_t launch_quantize8(const QuantParams& p, const QuantLaunch& l, cudaStream_t stream) {
@@ -715,9 +721,14 @@ cudaError_t launch_quantize8(const QuantParams& p, const QuantLaunch& l, cudaStr
   }
   const int tiles = l.tiles_q > l.tiles_k ? l.tiles_q : l.tiles_k;
   if (tiles == 0) return cudaSuccess;
-  dim3 g3(3 * tiles, p.Hq, p.B);
-  if (p.D == 64) quant8_kernel<64><<<g3, kThreads, 0, stream>>>(p);
-  else quant8_kernel<128><<<g3, kThreads, 0, stream>>>(p);
+  dim3 g3(2 * tiles, p.Hq, p.B);
+  if (p.D == 64) quant8_kernel<64, false><<<g3, kThreads, 0, stream>>>(p);
+  else quant8_kernel<128, false><<<g3, kThreads, 0, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || l.tiles_k == 0) return e;
+  dim3 g4(l.tiles_k, p.Hkv, p.B);
+  if (p.D == 64) quant8_kernel<64, true><<<g4, kThreads, 0, stream>>>(p);
+  else quant8_kernel<128, true><<<g4, kThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -746,9 +757,14 @@ cudaError_t launch_quantize(const QuantParams& p, const QuantLaunch& l, cudaStre
   }
   const int tiles = l.tiles_q > l.tiles_k ? l.tiles_q : l.tiles_k;
   if (tiles == 0) return cudaSuccess;
-  dim3 g3(3 * tiles, p.Hq, p.B);
-  if (p.D == 64) quant_kernel<64><<<g3, kThreads, 0, stream>>>(p);
-  else quant_kernel<128><<<g3, kThreads, 0, stream>>>(p);
+  dim3 g3(2 * tiles, p.Hq, p.B);
+  if (p.D == 64) quant_kernel<64, false><<<g3, kThreads, 0, stream>>>(p);
+  else quant_kernel<128, false><<<g3, kThreads, 0, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || l.tiles_k == 0) return e;
+  dim3 g4(l.tiles_k, p.Hkv, p.B);
+  if (p.D == 64) quant_kernel<64, true><<<g4, kThreads, 0, stream>>>(p);
+  else quant_kernel<128, true><<<g4, kThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
