@@ -11,17 +11,26 @@
 // key/value head h / (Hq / Hkv)), and the causal mask keeps key j <= i + (len_k - len_q)
 // for query i (the last query sees the last key). Warp roles:
 //   warp 0      TMA producer: Q^ + scales once, then K^/V^T tiles + scales into a
-//               3-stage shared-memory ring (cp.async.bulk.tensor / cp.async.bulk).
+//               4-stage shared-memory ring (cp.async.bulk.tensor / cp.async.bulk).
 //   warp 1      allocates 512 tensor-memory columns; one thread issues the tcgen05
 //               block-scaled MMAs: S = Q^ K^^T (kind::mxf4nvf4, M128 N128 K64 steps)
-//               into a double-buffered S in TMEM, and PV = P^ V^T (N = D) into TMEM.
-//   warps 2-9   two softmax/correction warpgroups. Thread (h, r) owns keys 64h..64h+63
-//               of query row r in every S tile and output channels [h*D/2, (h+1)*D/2)
-//               of that row. The two halves of a row exchange their maxima through
-//               shared memory; each half then computes P~, its per-16 E4M3 scales, the
-//               P^ codes (written in the swizzled layout the MMA reads) and its part of
-//               the row sum; and folds the previous tile's PV into its FP32 registers:
-//               O = O * alpha + s1 * PV.
+//               into S buffer j % 2, and PV = P^ V^T (N = D) into one PV accumulator,
+//               two key tiles behind the S products (the order in which they become
+//               ready when the two softmax warpgroups alternate).
+//   warps 2-3   idle (they complete the producer/MMA warpgroup, which gives registers
+//               to the correction warpgroup with setmaxnreg).
+//   warps 4-7   correction warpgroup. Thread r owns output row r in FP32 registers and
+//               folds every tile's PV row in: O = O * alpha + s1 * 2^(e - m_O) * PV,
+//               where e is the reference maximum the tile's softmax used and m_O its
+//               own reference.
+//   warps 8-15  two softmax warpgroups; warpgroup w takes key tiles j = w, w + 2, ...
+//               Thread r owns query row r of its tiles: it reads the 128 scores from
+//               TMEM (twice: block maxima first, then the exponentials), computes the
+//               tile maximum, P~, the per-16 E4M3 scales, the P^ codes (written in the
+//               swizzled layout the MMA reads) and the row sum relative to its own lazy
+//               reference maximum, and hands (reference, s1) to the correction. The
+//               two warpgroups never wait for each other, so one warpgroup's exp2 phase
+//               overlaps the other's TMEM loads, scales and barrier hand-offs.
 // Two instances per (D, causal): the general one (packed sequences, len_q != len_k,
 // second-level scales: per-sequence lengths, a mask offset, an empty-row guard and a
 // score scale read from the device) and a lean one for square dense problems with
@@ -47,10 +56,14 @@ using attn::store_out8;
 using attn::tmem_wait_regs;
 using attn::wait_bar;
 
-constexpr int kStages = 3;
-constexpr int kSoftmaxWarps = 8;
+constexpr int kStages = 4;
+constexpr int kCorrWarps = 4;      // warps 4-7
 constexpr uint32_t kTmemCols = 512;
-constexpr int kAttnThreads = 320;
+constexpr int kAttnThreads = 512;  // producer, MMA, 2 idle, 4 correction and 8 softmax warps
+// Per-thread registers after setmaxnreg: each SM sub-partition holds one warp of every
+// warpgroup, so 64 + 192 + 2 * 128 = 512 = 4 x the launch budget of 128.
+constexpr uint32_t kRegsLow = 64;
+constexpr uint32_t kRegsCorr = 192;
 
 constexpr int align1k(int x) { return (x + 1023) & ~1023; }
 
@@ -85,9 +98,9 @@ struct Layout {
   static constexpr int off_stage = align1k(off_sfq + kSfQKBytes);
   static constexpr int off_p = off_stage + kStages * kStageBytes;
   static constexpr int off_sfp = off_p + 2 * kPBytes;
-  static constexpr int off_xch = off_sfp + 2 * kSfPBytes;  // [2 tiles][2 halves][128] floats
-  static constexpr int off_lsum = off_xch + 2 * 2 * 128 * 4;  // [2 halves][128] floats
-  static constexpr int off_ones = align1k(off_lsum + 2 * 128 * 4);
+  static constexpr int off_info = off_sfp + 2 * kSfPBytes;  // [2 warpgroups][128] (reference, s1)
+  static constexpr int off_lsum = off_info + 2 * 128 * 8;    // [2 warpgroups][128] (l, reference)
+  static constexpr int off_ones = align1k(off_lsum + 2 * 128 * 8);
   static constexpr int off_bar = off_ones + kOnesBytes;
   static constexpr int kNumBars = 32;
   static constexpr int off_misc = off_bar + kNumBars * 8;    // tmem base, abort flag
@@ -106,8 +119,9 @@ enum : int {
   B_PEMPTY = B_PFULL + 2,
   B_PVFULL = B_PEMPTY + 2,
   B_PVEMPTY = B_PVFULL + 1,
-  B_XCH = B_PVEMPTY + 1,          // + tile parity: row-max exchange between the halves
-  B_LSUM = B_XCH + 2,             // final row-sum exchange
+  B_IFULL = B_PVEMPTY + 1,        // + softmax warpgroup: per-row factors of its latest tile
+  B_IEMPTY = B_IFULL + 2,
+  B_LSUM = B_IEMPTY + 2,          // final row sums of both softmax warpgroups
   B_DRAIN = B_LSUM + 1,
   B_COUNT = B_DRAIN + 1
 };
@@ -145,8 +159,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t bar0 = sbase + L::off_bar;
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + L::off_misc);
-  float* xch = reinterpret_cast<float*>(smem + L::off_xch);
-  float* lsum = reinterpret_cast<float*>(smem + L::off_lsum);
+  float2* info = reinterpret_cast<float2*>(smem + L::off_info);
+  float2* lsum = reinterpret_cast<float2*>(smem + L::off_lsum);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (seq_table_bad(p.seq)) return;
@@ -189,14 +203,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(B_SFULL + b), 1);
-      mbar_init(bar(B_SEMPTY + b), kSoftmaxWarps);
-      mbar_init(bar(B_PFULL + b), kSoftmaxWarps);
+      mbar_init(bar(B_SEMPTY + b), 4);
+      mbar_init(bar(B_PFULL + b), 4);
       mbar_init(bar(B_PEMPTY + b), 1);
-      mbar_init(bar(B_XCH + b), kSoftmaxWarps);
+      mbar_init(bar(B_IFULL + b), 4);
+      mbar_init(bar(B_IEMPTY + b), kCorrWarps);
     }
     mbar_init(bar(B_PVFULL), 1);
-    mbar_init(bar(B_PVEMPTY), kSoftmaxWarps);
-    mbar_init(bar(B_LSUM), kSoftmaxWarps);
+    mbar_init(bar(B_PVEMPTY), kCorrWarps);
+    mbar_init(bar(B_LSUM), 8);
     mbar_init(bar(B_DRAIN), 1);
     misc[1] = 0u;
     fence_mbar_init();
@@ -227,6 +242,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer ----
+    regs_decrease<kRegsLow>();
     if (lane == 0 && !(p.debug_flags & kDebugNoLoads)) {
       const uint32_t sq = sbase + L::off_q;
       mbar_arrive_expect_tx(bar(B_QFULL), L::kQBytes + L::kSfQKBytes);
@@ -264,6 +280,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer ----
+    regs_decrease<kRegsLow>();
     if (lane == 0) {
       constexpr uint32_t idesc_s = make_idesc_fp4(128);
       constexpr uint32_t idesc_pv = make_idesc_fp4(D);
@@ -274,7 +291,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int c = 0; c < kc_qk; ++c)
           tc_cp_sf(tmem + kColSfQ + 4 * c, sf_desc(sbase + L::off_sfq + 512 * c));
       }
-      for (int j = 0; ok && j <= nt; ++j) {
+      for (int j = 0; ok && j < nt + 2; ++j) {
         if (j < nt) {
           const int st = j % kStages, sb = j & 1;
           const uint32_t sst = sbase + L::off_stage + st * L::kStageBytes;
@@ -292,8 +309,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         make_sdesc(sst + L::st_bias, 128, 256, kLayoutNone), make_idesc_bf16(128), 1u);
           tc_commit(bar(B_SFULL + sb));
         }
-        if (j >= 1) {
-          const int jj = j - 1;
+        if (j >= 2) {
+          const int jj = j - 2;
           const int st = jj % kStages, pb = jj & 1;
           const uint32_t sst = sbase + L::off_stage + st * L::kStageBytes;
           if (!wait_bar(bar(B_VFULL + st), (jj / kStages) & 1, ctl)) { ok = false; break; }
@@ -319,196 +336,76 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       misc[3] = 0u;
       wait_bar(bar(B_DRAIN), 0, drain);
     }
-  } else {
-    // ------------------------------------------- softmax + correction (2 x 4 warps) ----
-    constexpr int DH = D / 2;
-    const int h = (warp - 2) >> 2;  // which half of the keys / output channels
-    const int quad = warp & 3;
+  } else if (warp < 4) {
+    regs_decrease<kRegsLow>();  // idle
+  } else if (warp < 4 + kCorrWarps) {
+    // ----------------------------------------------------- correction (4 warps) ----
+    regs_increase<kRegsCorr>();
+    constexpr int DH = D;
+    constexpr int cg = 0;
+    const int quad = warp & 3;       // TMEM lane quarter = rows 32*quad ..
     const int r = quad * 32 + lane;
     const int qrow = qt * 128 + r;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    float xs = p.sm_scale_log2, gv = 1.0f;
-    if (GENERAL && p.amax != nullptr) {
-      // Second-level scales fold into the score scale (Q and K) and the output (V).
-      const bool head = p.gscale == kGscaleHead;
-      const float gq = second_level_scale(p.amax[head ? bseq * p.Hq + hq : 0]);
-      const float gk = second_level_scale(p.amax[p.amax_stride + (head ? bseq * p.Hkv + hk : 0)]);
-      gv = second_level_scale(p.amax[2 * p.amax_stride + (head ? bseq * p.Hkv + hk : 0)]);
-      xs = xs * gq * gk;
-    }
+    float gv = 1.0f;
+    if (GENERAL && p.amax != nullptr)
+      gv = second_level_scale(p.amax[2 * p.amax_stride + (p.gscale == kGscaleHead ? bseq * p.Hkv + hk : 0)]);
     float o[DH];
 #pragma unroll
     for (int d = 0; d < DH; ++d) o[d] = 0.0f;
-    float m_run = -INFINITY, l_half = 0.0f, alpha_prev = 1.0f, s1_prev = 0.0f;
+    // O is kept relative to 2^m_o; m_o moves (and O is rescaled) only when a tile's
+    // reference exceeds it by more than 8, so the factor 2^(e - m_o) stays <= 2^8.
+    float m_o = -INFINITY;
     bool ok = true;
-
-    // O = O * alpha + s1 * PV for this thread's DH output channels (PV of tile jj).
-    auto correct = [&](int jj, float alpha, float s1) -> bool {
-      if (!__all_sync(0xffffffffu, wait_bar(bar(B_PVFULL), jj & 1, ctl))) return false;
+    for (int j = 0; j < nt; ++j) {
+      const int w = j & 1;
+      if (!__all_sync(0xffffffffu, wait_bar(bar(B_IFULL + w), (j >> 1) & 1, ctl))) { ok = false; break; }
+      const float2 f = info[w * 128 + r];  // (reference e, s1) of tile j for this row
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_IEMPTY + w));
+      float alpha = 1.0f, c = 0.0f;
+      if (f.y > 0.0f) {  // s1 = 0: the row saw no key of this tile
+        if (f.x > m_o + 8.0f) {
+          alpha = ex2_approx(m_o - f.x);  // 0 on the first contribution (m_o = -inf)
+          m_o = f.x;
+        }
+        c = f.y * ex2_approx(f.x - m_o);
+      }
+      if (!__all_sync(0xffffffffu, wait_bar(bar(B_PVFULL), j & 1, ctl))) { ok = false; break; }
       tc_fence_after();
       const bool unit = __all_sync(0xffffffffu, alpha == 1.0f);
+      const float2 c2 = make_float2(c, c), a2 = make_float2(alpha, alpha);
 #pragma unroll
-      for (int c = 0; c < DH / 32; ++c) {
+      for (int cc = 0; cc < DH / 32; ++cc) {
         uint32_t v[32];
-        tmem_ld32(tmem + lane_base + kColPV + DH * h + 32 * c, v);
+        tmem_ld32(tmem + lane_base + kColPV + DH * cg + 32 * cc, v);
         tmem_wait_regs(v);
-        const float2 s12 = make_float2(s1, s1), a2 = make_float2(alpha, alpha);
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          float2 acc = make_float2(o[32 * c + i], o[32 * c + i + 1]);
+          float2 acc = make_float2(o[32 * cc + i], o[32 * cc + i + 1]);
           if (!unit) acc = mul2(acc, a2);
-          acc = fma2(make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), s12, acc);
-          o[32 * c + i] = acc.x;
-          o[32 * c + i + 1] = acc.y;
+          acc = fma2(make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), c2, acc);
+          o[32 * cc + i] = acc.x;
+          o[32 * cc + i + 1] = acc.y;
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_PVEMPTY));
-      return true;
-    };
-
-    for (int j = 0; j < nt; ++j) {
-      const int sb = j & 1, pb = j & 1;
-      if (!__all_sync(0xffffffffu, wait_bar(bar(B_SFULL + sb), (j >> 1) & 1, ctl))) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sr[2][32];
-      tmem_ld32(tmem + lane_base + kColS0 + 128 * sb + 64 * h, sr[0]);
-      tmem_ld32(tmem + lane_base + kColS0 + 128 * sb + 64 * h + 32, sr[1]);
-      tmem_wait_regs(sr[0]);
-      tmem_wait_regs(sr[1]);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_SEMPTY + sb));
-
-      float s[64];
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(sr[c][i]);
-      const int kbase = j * 128 + 64 * h;
-      const bool need_mask = GENERAL ? ((j * 128 + 128 > si.len_k) || (CAUSAL && j * 128 + 127 > qt * 128 + coff))
-                                     : (CAUSAL ? (j == nt - 1) : (j * 128 + 128 > p.seq.Nk));
-      if (need_mask) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int key = kbase + c;
-          if (GENERAL ? (key >= si.len_k || (CAUSAL && key > qrow + coff))
-                      : (key >= p.seq.Nk || (CAUSAL && key > qrow)))
-            s[c] = -INFINITY;
-        }
-      }
-      // Block maxima of the raw scores (sm_scale > 0, so they order like P~).
-      float bm[4];
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        float m0 = max3(s[16 * b], s[16 * b + 1], s[16 * b + 2]);
-#pragma unroll
-        for (int i = 3; i < 15; i += 2) m0 = max3(m0, s[16 * b + i], s[16 * b + i + 1]);
-        bm[b] = fmaxf(m0, s[16 * b + 15]);
-      }
-      const float hm = fmaxf(fmaxf(bm[0], bm[1]), fmaxf(bm[2], bm[3]));
-      float* xb = xch + (j & 1) * 256;
-      xb[h * 128 + r] = hm;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_XCH + (j & 1)));
-      if (!__all_sync(0xffffffffu, wait_bar(bar(B_XCH + (j & 1)), (j >> 1) & 1, ctl))) { ok = false; break; }
-      const float tm = fmaxf(hm, xb[(1 - h) * 128 + r]);
-      // A row can see no key of this tile (causal with len_q > len_k, or a mask offset
-      // that is not a multiple of 128): it then adds nothing, and its P^ codes are 0.
-      const bool empty = GENERAL && tm == -INFINITY;
-
-      const float tmx = tm * xs;
-      // Reference max: it moves only when the tile max exceeds it by more than 8 (log2
-      // units). The reference cancels in O / l, and the P~ quantization below is relative
-      // to the tile max, so this changes rounding only while the O rescale is skipped on
-      // most tiles.
-      const bool move = tmx > m_run + 8.0f;  // always true on the first tile (m_run = -inf)
-      const float m_new = move ? tmx : m_run;
-      const float alpha = move ? ex2_approx(m_run - m_new) : 1.0f;
-      const float rfac = empty ? 0.0f : ex2_approx(tmx - m_new);  // rowmax of P~ in this tile (<= 2^8)
-      const float s1 = rfac * (1.0f / 2688.0f);
-      const float tref = empty ? 0.0f : tmx;
-
-      // Per-16 scales of P2 = P~ / s1 = exp2(S*xs - tmx) * 2688. The division by the
-      // decoded block scale is folded into the exp2 argument: v = exp2(S*xs - nb) = P2 / s.
-      // A block whose scale rounds to zero keeps the plain exp2 (for the row sum) and
-      // gets zero codes.
-      float nb[4], mult[4];
-      uint32_t sfw = 0, zero_blocks = 0;
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const float amax = ex2_approx(fmaf(bm[b], xs, -tref)) * 2688.0f;
-        const uint32_t sbyte = f32_to_e4m3(amax * (1.0f / 6.0f));
-        const float sdec = e4m3_to_f32(sbyte);
-        if (sdec > 0.0f) {
-          nb[b] = -(tref + lg2_approx(sdec) - 11.392317422778761f);  // log2(2688)
-          mult[b] = sdec * (1.0f / 2688.0f);
-        } else {
-          nb[b] = -tref;
-          mult[b] = 1.0f;
-          zero_blocks |= 1u << b;
-        }
-        sfw |= sbyte << (8 * b);
-      }
-      float rsum = 0.0f;
-      uint32_t pw[8];
-      const float2 xs2 = make_float2(xs, xs);
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const float2 nb2 = make_float2(nb[b], nb[b]);
-        float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-          float e[8];
-#pragma unroll
-          for (int q2 = 0; q2 < 4; ++q2) {
-            const int k0 = 16 * b + 8 * w + 2 * q2;
-            const float2 arg = fma2(make_float2(s[k0], s[k0 + 1]), xs2, nb2);
-            const float2 ee = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
-            acc = add2(acc, ee);
-            e[2 * q2] = ee.x;
-            e[2 * q2 + 1] = ee.y;
-          }
-          const uint32_t word = f32x8_to_e2m1(e[0], e[1], e[2], e[3], e[4], e[5], e[6], e[7]);
-          pw[2 * b + w] = (zero_blocks >> b) & 1u ? 0u : word;
-        }
-        rsum += (acc.x + acc.y) * mult[b];
-      }
-      l_half = l_half * alpha + rsum * rfac;
-      m_run = m_new;
-
-      // P^ buffer pb must be free (PV of tile j-2 finished).
-      if (!__all_sync(0xffffffffu, wait_bar(bar(B_PEMPTY + pb), ((j >> 1) & 1) ^ 1, ctl))) { ok = false; break; }
-      uint8_t* prow = smem + L::off_p + pb * L::kPBytes + r * 64;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int cs = (2 * h + c) ^ ((r >> 1) & 3);
-        *reinterpret_cast<uint4*>(prow + cs * 16) =
-            make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-      }
-      *reinterpret_cast<uint32_t*>(smem + L::off_sfp + pb * L::kSfPBytes + 512 * h + (r % 32) * 16 + (r / 32) * 4) = sfw;
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_PFULL + pb));
-
-      if (j >= 1 && !correct(j - 1, alpha_prev, s1_prev)) { ok = false; break; }
-      alpha_prev = alpha;
-      s1_prev = s1;
     }
-    if (ok && nt > 0) ok = correct(nt - 1, alpha_prev, s1_prev);
-    if (ok) {
-      lsum[h * 128 + r] = l_half;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_LSUM));
-      ok = __all_sync(0xffffffffu, wait_bar(bar(B_LSUM), 0, ctl));
-    }
+    if (ok) ok = __all_sync(0xffffffffu, wait_bar(bar(B_LSUM), 0, ctl));
     if (ok && qrow < si.len_q) {
-      // A row that saw no key (l = 0) is written as 0.
-      const float l = l_half + lsum[(1 - h) * 128 + r];
+      // l = sum over the two softmax warpgroups of l_w * 2^(m_w - m_o); a row that saw
+      // no key (l = 0) is written as 0.
+      float l = 0.0f;
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        const float2 e = lsum[w * 128 + r];
+        if (e.x > 0.0f) l += e.x * ex2_approx(e.y - m_o);
+      }
       const float il = l > 0.0f ? gv / l : 0.0f;
       const size_t base = static_cast<size_t>(static_cast<int64_t>(bseq) * p.so.b + static_cast<int64_t>(hq) * p.so.h +
-                                              (static_cast<int64_t>(si.tok_q) + qrow) * p.so.n) + DH * h;
+                                              (static_cast<int64_t>(si.tok_q) + qrow) * p.so.n) + DH * cg;
 #pragma unroll
       for (int d = 0; d < DH; d += 8) {
         float v8[8];
@@ -516,6 +413,162 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int i = 0; i < 8; ++i) v8[i] = o[d + i] * il;
         store_out8(p.out, base + d, v8, p.out_dtype);
       }
+    }
+  } else {
+    // ----------------------------------------------------- softmax (2 x 4 warps) ----
+    const int sw = (warp - 4 - kCorrWarps) >> 2;  // key tiles j = sw, sw + 2, ...
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int qrow = qt * 128 + r;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    float xs = p.sm_scale_log2;
+    if (GENERAL && p.amax != nullptr) {
+      // Second-level scales of Q and K fold into the score scale.
+      const bool head = p.gscale == kGscaleHead;
+      const float gq = second_level_scale(p.amax[head ? bseq * p.Hq + hq : 0]);
+      const float gk = second_level_scale(p.amax[p.amax_stride + (head ? bseq * p.Hkv + hk : 0)]);
+      xs = xs * gq * gk;
+    }
+    const float2 xs2 = make_float2(xs, xs);
+    float m_w = -INFINITY, l_w = 0.0f;
+    bool ok = true;
+    uint8_t* prow = smem + L::off_p + sw * L::kPBytes + r * 64;
+    uint8_t* sfrow = smem + L::off_sfp + sw * L::kSfPBytes + (r % 32) * 16 + (r / 32) * 4;
+    const uint32_t scol = tmem + lane_base + kColS0 + 128 * sw;
+
+    for (int j = sw; j < nt; j += 2) {
+      const int use = j >> 1;  // use count of S / P buffer sw
+      if (!__all_sync(0xffffffffu, wait_bar(bar(B_SFULL + sw), use & 1, ctl))) { ok = false; break; }
+      tc_fence_after();
+      const int kbase = j * 128;
+      const bool need_mask = GENERAL ? ((j * 128 + 128 > si.len_k) || (CAUSAL && j * 128 + 127 > qt * 128 + coff))
+                                     : (CAUSAL ? (j == nt - 1) : (j * 128 + 128 > p.seq.Nk));
+      // Scores of keys k0 .. k0 + 31 as floats, masked keys -> -inf.
+      auto load_mask = [&](uint32_t (&v)[32], int k0) {
+        if (need_mask) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int key = kbase + k0 + i;
+            if (GENERAL ? (key >= si.len_k || (CAUSAL && key > qrow + coff))
+                        : (key >= p.seq.Nk || (CAUSAL && key > qrow)))
+              v[i] = __float_as_uint(-INFINITY);
+          }
+        }
+      };
+      auto block_max16 = [&](const uint32_t (&v)[32], int i0) {
+        float m0 = max3(__uint_as_float(v[i0]), __uint_as_float(v[i0 + 1]), __uint_as_float(v[i0 + 2]));
+#pragma unroll
+        for (int i = 3; i < 15; i += 2) m0 = max3(m0, __uint_as_float(v[i0 + i]), __uint_as_float(v[i0 + i + 1]));
+        return fmaxf(m0, __uint_as_float(v[i0 + 15]));
+      };
+      // Pass 1: block maxima of the raw scores (sm_scale > 0, so they order like P~).
+      uint32_t sa[32], sb[32];
+      float bm[8];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        tmem_ld32(scol + 64 * hh, sa);
+        tmem_ld32(scol + 64 * hh + 32, sb);
+        tmem_wait_regs(sa);
+        tmem_wait_regs(sb);
+        load_mask(sa, 64 * hh);
+        load_mask(sb, 64 * hh + 32);
+        bm[4 * hh] = block_max16(sa, 0);
+        bm[4 * hh + 1] = block_max16(sa, 16);
+        bm[4 * hh + 2] = block_max16(sb, 0);
+        bm[4 * hh + 3] = block_max16(sb, 16);
+      }
+      const float tm = fmaxf(fmaxf(max3(bm[0], bm[1], bm[2]), max3(bm[3], bm[4], bm[5])), fmaxf(bm[6], bm[7]));
+      // A row can see no key of this tile (causal with len_q > len_k, or a mask offset
+      // that is not a multiple of 128): it then adds nothing, and its P^ codes are 0.
+      const bool empty = GENERAL && tm == -INFINITY;
+      const float tmx = tm * xs;
+      // Lazy reference maximum: it moves only when the tile maximum exceeds it by more
+      // than 8 (log2 units). It cancels in O / l, and P~ is quantized relative to the
+      // tile maximum, so it only decides how often l and O are rescaled.
+      const bool move = tmx > m_w + 8.0f;  // always true on the first tile (m_w = -inf)
+      const float m_new = move ? tmx : m_w;
+      const float alpha = move ? ex2_approx(m_w - m_new) : 1.0f;
+      const float rfac = empty ? 0.0f : ex2_approx(tmx - m_new);  // rowmax of P~ in this tile (<= 2^8)
+      const float tref = empty ? 0.0f : tmx;
+      // Per-16 scales of P2 = P~ / s1 = exp2(S*xs - tmx) * 2688 (E4M3 of blockmax / 6).
+      uint32_t sfw[2] = {0u, 0u};
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        const float amax = ex2_approx(fmaf(bm[b], xs, -tref)) * 2688.0f;
+        sfw[b >> 2] |= f32_to_e4m3(amax * (1.0f / 6.0f)) << (8 * (b & 3));
+      }
+      // P^ buffer sw must be free (PV of tile j - 2 finished).
+      if (!__all_sync(0xffffffffu, wait_bar(bar(B_PEMPTY + sw), (use & 1) ^ 1, ctl))) { ok = false; break; }
+      float rsum = 0.0f;
+      // Codes of keys 32c .. 32c + 31. The division by the decoded block scale is folded
+      // into the exp2 argument: v = exp2(S*xs - nb) = P2 / s. A block whose scale rounds
+      // to zero keeps the plain exp2 (for the row sum) and gets zero codes.
+      auto emit = [&](const uint32_t (&v)[32], int c) {
+        uint32_t pw[4];
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const int b = 2 * c + bb;
+          const uint32_t sbyte = (sfw[b >> 2] >> (8 * (b & 3))) & 0xFFu;
+          float nb = -tref, mult = 1.0f;
+          if (sbyte != 0u) {
+            const float sdec = e4m3_to_f32(sbyte);
+            nb = -(tref + lg2_approx(sdec) - 11.392317422778761f);  // log2(2688)
+            mult = sdec * (1.0f / 2688.0f);
+          }
+          const float2 nb2 = make_float2(nb, nb);
+          float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            float e[8];
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
+              const int k0 = 16 * bb + 8 * w + 2 * q2;
+              const float2 arg = fma2(make_float2(__uint_as_float(v[k0]), __uint_as_float(v[k0 + 1])), xs2, nb2);
+              const float2 ee = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+              acc = add2(acc, ee);
+              e[2 * q2] = ee.x;
+              e[2 * q2 + 1] = ee.y;
+            }
+            const uint32_t word = f32x8_to_e2m1(e[0], e[1], e[2], e[3], e[4], e[5], e[6], e[7]);
+            pw[2 * bb + w] = sbyte != 0u ? word : 0u;
+          }
+          rsum += (acc.x + acc.y) * mult;
+        }
+        *reinterpret_cast<uint4*>(prow + ((c ^ ((r >> 1) & 3)) * 16)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+      };
+      // Pass 2: keys 64-127 are still in registers; keys 0-63 are read again, after
+      // which the S buffer goes back to the MMA warp.
+      emit(sa, 2);
+      emit(sb, 3);
+      tmem_ld32(scol, sa);
+      tmem_ld32(scol + 32, sb);
+      tmem_wait_regs(sa);
+      tmem_wait_regs(sb);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_SEMPTY + sw));
+      load_mask(sa, 0);
+      load_mask(sb, 32);
+      emit(sa, 0);
+      emit(sb, 1);
+      *reinterpret_cast<uint32_t*>(sfrow) = sfw[0];
+      *reinterpret_cast<uint32_t*>(sfrow + 512) = sfw[1];
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_PFULL + sw));
+
+      // (reference, s1) of this tile for the correction warpgroups.
+      if (!__all_sync(0xffffffffu, wait_bar(bar(B_IEMPTY + sw), (use & 1) ^ 1, ctl))) { ok = false; break; }
+      info[sw * 128 + r] = make_float2(m_new, rfac * (1.0f / 2688.0f));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_IFULL + sw));
+      l_w = l_w * alpha + rsum * rfac;
+      m_w = m_new;
+    }
+    if (ok) {
+      lsum[sw * 128 + r] = make_float2(l_w, m_w);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_LSUM));
     }
   }
 
