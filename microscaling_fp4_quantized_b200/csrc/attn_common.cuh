@@ -19,12 +19,28 @@ struct Ctl {
   uint64_t timeout_ns;
 };
 
+// Suspend bound of one try_wait for threads that let themselves be suspended while they
+// wait.
+constexpr uint32_t kSuspendNs = 500;
+
+__device__ __forceinline__ bool try_wait_for(uint32_t bar, uint32_t parity, uint32_t sleep_ns) {
+  return sleep_ns != 0u ? mbar_try_wait_sleep(bar, parity, sleep_ns) : mbar_try_wait(bar, parity);
+}
+
 // Bounded wait: true when the phase with `parity` has completed, false on abort/timeout.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& c) {
-  if (mbar_try_wait(bar, parity)) return true;
+// sleep_ns != 0 lets the thread stay suspended in each probe for up to that long; the
+// abort flag and the clock are read after every probe whose index & check_mask is 0.
+// Measured on the FP4 attention kernel: its non-causal instances run fastest with
+// suspended probes and a check after each, the causal ones with plain probes and a
+// check every 32nd (per-tile times 1110 vs 1225 ns on long non-causal rows, 1413 vs
+// 1785 ns on causal ones).
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& c, uint32_t sleep_ns = 0u,
+                                         uint32_t check_mask = 0u) {
+  if (try_wait_for(bar, parity, sleep_ns)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+  for (uint32_t it = 1;; ++it) {
+    if (try_wait_for(bar, parity, sleep_ns)) return true;
+    if ((it & check_mask) != 0u) continue;
     if (*c.abort) return false;
     if (globaltimer_ns() - t0 > c.timeout_ns) {
       *c.abort = 1u;
