@@ -103,14 +103,18 @@ class ClockSampler:
 
 def _attn_traffic(wl, b8=False):
     """DRAM bytes per attention launch from the committed ncu capture, or None when the
-    kernel source has changed since the capture (or no capture exists)."""
+    kernel sources (hashed in the record's order) have changed since the capture, or
+    no capture exists."""
     import hashlib
     name = "attn8_fwd_kernel_traffic.json" if b8 else "attn_fp4_fwd_kernel_traffic.json"
     try:
         with open(os.path.join(ROOT, "profiles", name)) as f:
             rec = json.load(f)
-        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
+        h = hashlib.sha256()
+        for src in rec.get("sources") or [rec["source"]]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        sha = h.hexdigest()
     except Exception:
         return None, "no capture"
     if not sha.startswith(rec["source_sha256_prefix"]):
