@@ -118,3 +118,37 @@ def test_argument_errors(sage):
     with pytest.raises(sage.SageError) as e:
         sage.attn(mis, mis, mis)
     assert e.value.status == sage.SAGE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+def test_attn_alternating_tile_maxima(sage, oracle_mod, causal):
+    """Key tiles whose score level alternates between far above and far below the others
+    (plus a drift across tiles): consecutive key tiles go to different softmax warpgroups,
+    so their lazy reference maxima differ by far more than the rescale threshold and the
+    correction re-bases every tile's contribution and moves its own reference often."""
+    B, H, N, D = 1, 2, 1280, 128
+    g = torch.Generator(device="cpu")
+    g.manual_seed(61)
+    u = torch.randn(D, generator=g)
+    u = u / u.norm()
+    q = torch.randn((B, H, N, D), generator=g) * 0.5 + 3.0 * u
+    k = torch.randn((B, H, N, D), generator=g) * 0.5
+    v = torch.randn((B, H, N, D), generator=g)
+    tiles = torch.arange(N) // 128
+    level = torch.where(tiles % 2 == 0, 1.0, -1.0) * 20.0 + 2.5 * tiles.float()
+    k = k + level[None, None, :, None] * u
+    q, k, v = (t.to(torch.bfloat16).cuda() for t in (q, k, v))
+    sm = 1.0 / np.sqrt(D)
+    out = sage.attn(q, k, v, causal=causal, sm_scale=sm)
+    torch.cuda.synchronize()
+    assert sage.device_error() == 0
+    hs = list(range(B * H))
+    qo, ko, vo = heads_view(q, hs), heads_view(k, hs), heads_view(v, hs)
+    got = f32(out.reshape(B * H, N, D)).reshape(-1, D)
+    assert np.isfinite(got).all()
+    em, _ = oracle_mod.attention(qo, ko, vo, causal, sm, Bk=128)
+    m_em = oracle_mod.metrics(got, em.reshape(-1, D))
+    vmax = float(np.abs(vo).max())
+    print(f"\nalternating tile maxima ({'causal' if causal else 'full'}): vs emulated {m_em}")
+    assert m_em["max_abs"] <= MAX_ABS_FRAC * vmax, m_em
+    assert m_em["cos"] >= MIN_COS, m_em
