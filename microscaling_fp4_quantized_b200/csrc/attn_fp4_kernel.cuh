@@ -36,11 +36,12 @@
 //               reference maximum, and hands (reference, s1) to the correction. The
 //               two warpgroups never wait for each other, so one warpgroup's exp2 phase
 //               overlaps the other's TMEM loads, scales and barrier hand-offs.
-// Two instances per (D, causal): the general one (packed sequences, len_q != len_k,
+// Three instances per (D, causal): the general one (packed sequences, len_q != len_k,
 // second-level scales: per-sequence lengths, a mask offset, an empty-row guard and a
-// score scale read from the device) and a lean one for square dense problems with
-// one-level scales, whose loop keeps the score scale and the lengths as kernel
-// parameters (about 1.5 % faster on the long non-causal workload).
+// score scale read from the device), the general one with the Q-smoothing bias MMA, and
+// a lean one for square dense problems with one-level scales, whose loop keeps the score
+// scale and the lengths as kernel parameters (long non-causal workload: 1163 TFLOP/s
+// lean, 1051 general with a per-tensor second-level scale).
 // Every mbarrier wait is bounded (globaltimer); a wait that runs out raises the CTA's
 // abort flag and the device error word, and all roles drain and return.
 #pragma once
