@@ -70,9 +70,15 @@ __device__ __forceinline__ bool seq_table_bad(const SeqMap& m) {
   return m.bad != nullptr && *reinterpret_cast<const volatile uint32_t*>(m.bad) != 0u;
 }
 
-// Second-level scale from a group maximum: fp32(amax / 2688), or 1 when that is 0.
+// Second-level scale from a group maximum: fp32(amax / 2688), or 1 when that is 0. The
+// quotient is the double product amax * RN64(1/2688) rounded to binary32, which equals the
+// IEEE binary32 division for every non-negative binary32 amax (checked exhaustively on the
+// CPU: the exact quotient's binary fraction repeats with period 6, 2688 = 21 * 2^7, so it
+// never lies within the double product's error of a binary32 rounding midpoint). It keeps
+// the division's subroutine out of the attention kernel (measured 1053 -> 1082 TFLOP/s for
+// its general instance on the long workload).
 __device__ __forceinline__ float second_level_scale(float amax) {
-  const float g = __fdiv_rn(amax, kTwoLevelTarget);
+  const float g = __double2float_rn(static_cast<double>(amax) * (1.0 / 2688.0));
   return g > 0.0f ? g : 1.0f;
 }
 

@@ -5,7 +5,11 @@
  *   - for every positive finite E4M3 divisor and every |x / d| in [2^-4, 2^4), visiting
  *     every `stride`-th binary32 x (stride 1 = exhaustive), both signs, and x = -0;
  *   - for d = 6 and every `stride`-th positive binary32 x whose quotient is normal.
- * Prints the number of mismatches of each part; exit status 0 when both are 0. */
+ * And the one the second-level scale relies on: for every `stride`-th non-negative finite
+ * binary32 x, fp32(double(x) * RN64(1/2688)) equals the IEEE binary32 quotient x / 2688
+ * (the exact quotient's binary fraction repeats with period 6 -- 2688 = 21 * 2^7 -- so it
+ * is never within 2^-52 of a binary32 rounding midpoint; subnormal quotients included).
+ * Prints the number of mismatches of each part; exit status 0 when all are 0. */
 #include <math.h>
 #include <stdint.h>
 #include <stdio.h>
@@ -50,6 +54,16 @@ int main(int argc, char** argv) {
     if (u_of(div_fma(a, 6.0f, r6)) != u_of(a / 6.0f)) ++bad6;
     ++n6;
   }
-  printf("e4m3 divisors: %ld checks, %ld mismatches; d = 6: %ld checks, %ld mismatches\n", n, bad, n6, bad6);
-  return (bad == 0 && bad6 == 0) ? 0 : 1;
+  long n2688 = 0, bad2688 = 0;
+  const double c2688 = 1.0 / 2688.0;
+  for (uint32_t u = 0; u < 0x7F800000u; u += stride) {  /* second-level scale: x / 2688 */
+    const float x = f_of(u);
+    volatile float ref = x / 2688.0f;
+    const float got = (float)((double)x * c2688);
+    ++n2688;
+    if (u_of(ref) != u_of(got)) ++bad2688;
+  }
+  printf("e4m3 divisors: %ld checks, %ld mismatches; d = 6: %ld checks, %ld mismatches; "
+         "x / 2688 by a double product: %ld checks, %ld mismatches\n", n, bad, n6, bad6, n2688, bad2688);
+  return (bad == 0 && bad6 == 0 && bad2688 == 0) ? 0 : 1;
 }

@@ -1,8 +1,8 @@
 """The quantization kernel divides by E4M3 block scales and by 6 with Markstein's
-FMA-corrected quotient instead of a full IEEE division. This checks, on the CPU, that
-the identity holds on the domain where the E2M1 code or E4M3 scale byte depends on the
-last bit of the quotient (a strided subset here; the exhaustive run, stride 1, also
-passes)."""
+FMA-corrected quotient instead of a full IEEE division, and the second-level scale
+amax / 2688 is a double-precision product rounded to binary32. This checks, on the CPU,
+that the identities hold on the domains the kernels use them on (a strided subset here;
+the exhaustive run, stride 1, also passes)."""
 import os
 import subprocess
 
