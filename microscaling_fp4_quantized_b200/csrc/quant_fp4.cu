@@ -14,8 +14,9 @@
 // of K first. The optional second-level scale (NVFP4's FP32 factor, named on the
 // author page, "TetraJet-v2" abstract) divides a whole tensor, or one head of one
 // sequence, by g = amax / 2688 before the block rule -- the same two-level shape the
-// method gives P~. Every arithmetic step is IEEE binary32 with RNE (true divisions, no
-// reciprocal), so codes and scale bytes are reproducible bit for bit.
+// method gives P~. Every arithmetic step is IEEE binary32 with RNE, and every quotient is
+// the IEEE binary32 quotient (an IEEE division, or one of the two forms below proven to
+// equal it where they are used), so codes and scale bytes are reproducible bit for bit.
 //
 // All four kernels are HBM-bound (or tiny): 16-byte coalesced loads, tiles of 128
 // tokens, scale factors and V^T codes staged in shared memory and written out as
@@ -66,6 +67,31 @@ __device__ __forceinline__ float div_fma(float x, float d, float r) {
   const float q = __fmul_rn(x, r);
   const float e = __fmaf_rn(-q, d, x);
   return copysignf(__fmaf_rn(e, r, q), x);
+}
+
+// x / d rounded to binary32 exactly as the IEEE division, from c ~ 1/d in double formed
+// once per divisor (recip_d): the double product x * c is within ~2^-52 (relative) of
+// x / d, while for binary32 x and d the quotient is either representable or at least
+// 2^-49 (relative) away from every binary32 rounding midpoint (x - d * mid is a nonzero
+// multiple of ulp(d) * ulp(mid) / 2, and a midpoint has 25 significant bits), so rounding
+// the product gives the correctly rounded quotient -- subnormal quotients included.
+// Checked on the CPU for random divisors with the same reciprocal sequence.
+__device__ __forceinline__ float div_by(float x, double c) {
+  return __double2float_rn(static_cast<double>(x) * c);
+}
+
+// 1/d in double to ~2^-53 relative for a positive finite binary32 d: the binary32
+// reciprocal refined by two Newton steps (each squares the relative error) in double
+// FMAs; d below 2^-64 is scaled by 2^64 first so that the binary32 reciprocal stays
+// finite. No division, so no division subroutine in the kernel.
+__device__ __forceinline__ double recip_d(float d) {
+  const bool tiny = d < 5.421010862427522e-20f;  // 2^-64
+  const float ds = tiny ? d * 18446744073709551616.0f : d;
+  const double dd = static_cast<double>(ds);
+  double y = static_cast<double>(__frcp_rn(ds));
+  y = fma(y, fma(-dd, y, 1.0), y);
+  y = fma(y, fma(-dd, y, 1.0), y);
+  return tiny ? y * 18446744073709551616.0 : y;
 }
 
 // RN(1/6) in binary32.
@@ -386,7 +412,7 @@ __global__ void __launch_bounds__(D) finalize_kernel(QuantParams p) {
 // At most 64 registers (4 CTAs per SM): the extra resident warps hide more load latency
 // than the few spilled values cost (measured 0.35 -> 0.31 ms for the long workload's
 // quantization with the statistics loop unrolled 8-deep; identical output bytes).
-template <int D, bool VJOB>
+template <int D, bool VJOB, bool GS>
 __global__ void __launch_bounds__(kThreads, 4) quant_kernel(QuantParams p) {
   constexpr int CPR = D / 8;
   constexpr int kVRowBytes = (D + 8) * 2;  // padded V tile row (16-byte multiple)
@@ -409,9 +435,10 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(QuantParams p) {
   const int64_t row0 = static_cast<int64_t>(H) * prow + static_cast<int64_t>(h) * ntile * 128 + tile * 128;
   const int64_t T = row0 >> 7;  // scale-factor / V^T tile index
   const int rows = min(128, len - tile * 128);
-  const bool gs = p.gscale != kGscaleNone;
+  constexpr bool gs = GS;  // second-level scale (its own instance, so the plain one carries none of its code)
   float g = 1.0f;
   if (gs) g = second_level_scale(p.amax[job * p.amax_stride + (p.gscale == kGscaleHead ? b * H + h : 0)]);
+  const double cg = gs ? recip_d(g) : 1.0;  // x / g = div_by(x, cg)
 
   if constexpr (!VJOB) {
     uint8_t* sfbuf = smem;                                  // kSfBytesQK
@@ -489,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(QuantParams p) {
       }
       if (rl < rows && gs) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = __fdiv_rn(x[e], g);
+        for (int e = 0; e < 8; ++e) x[e] = div_by(x[e], cg);
       }
       float a = 0.0f;
 #pragma unroll
@@ -536,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(QuantParams p) {
         const uint16_t hv = *reinterpret_cast<const uint16_t*>(vtile + (tb * 16 + i) * kVRowBytes + d * 2);
         x[i] = (p.dtype == kDtypeBF16) ? __uint_as_float(static_cast<uint32_t>(hv) << 16)
                                        : __half2float(__ushort_as_half(hv));
-        if (gs) x[i] = __fdiv_rn(x[i], g);
+        if (gs) x[i] = div_by(x[i], cg);
       }
       float a = 0.0f;
   #pragma unroll
@@ -635,6 +662,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant8_kernel(QuantParams p) {
     }
     a = block_max(a, redw);
     const float s = __fdiv_rn(a, 127.0f);
+    const double cs = s > 0.0f ? recip_d(s) : 0.0;  // x / s = div_by(x, cs)
     if (t == 0) reinterpret_cast<float*>(job == 0 ? p.q_sf : p.k_sf)[T] = s;
     uint8_t* dst = (job == 0 ? p.q_fp4 : p.k_fp4) + row0 * D;
 #pragma unroll
@@ -645,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant8_kernel(QuantParams p) {
       if (s > 0.0f) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float r = fminf(127.0f, fmaxf(-127.0f, rintf(__fdiv_rn(x[e], s))));
+          const float r = fminf(127.0f, fmaxf(-127.0f, rintf(div_by(x[e], cs))));
           w[e >> 2] |= (static_cast<uint32_t>(static_cast<int>(r)) & 0xFFu) << (8 * (e & 3));
         }
       }
@@ -675,6 +703,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant8_kernel(QuantParams p) {
     const int item = t + k * kThreads;
     const int d = item % D, tb = item / D;
     const float s = sv[d];
+    const double cs = s > 0.0f ? recip_d(s) : 0.0;  // x / s = div_by(x, cs)
     uint32_t w[4] = {0u, 0u, 0u, 0u};
     if (s > 0.0f) {
 #pragma unroll
@@ -682,7 +711,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant8_kernel(QuantParams p) {
         const uint16_t hv = *reinterpret_cast<const uint16_t*>(vtile + (tb * 16 + i) * kVRowBytes + d * 2);
         const float x = (p.dtype == kDtypeBF16) ? __uint_as_float(static_cast<uint32_t>(hv) << 16)
                                                 : __half2float(__ushort_as_half(hv));
-        w[i >> 2] |= f32_to_e4m3(__fdiv_rn(x, s)) << (8 * (i & 3));
+        w[i >> 2] |= f32_to_e4m3(div_by(x, cs)) << (8 * (i & 3));
       }
     }
     codes[k] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -763,13 +792,23 @@ cudaError_t launch_quantize(const QuantParams& p, const QuantLaunch& l, cudaStre
   const int tiles = l.tiles_q > l.tiles_k ? l.tiles_q : l.tiles_k;
   if (tiles == 0) return cudaSuccess;
   dim3 g3(2 * tiles, p.Hq, p.B);
-  if (p.D == 64) quant_kernel<64, false><<<g3, kThreads, 0, stream>>>(p);
-  else quant_kernel<128, false><<<g3, kThreads, 0, stream>>>(p);
+  if (gs) {
+    if (p.D == 64) quant_kernel<64, false, true><<<g3, kThreads, 0, stream>>>(p);
+    else quant_kernel<128, false, true><<<g3, kThreads, 0, stream>>>(p);
+  } else {
+    if (p.D == 64) quant_kernel<64, false, false><<<g3, kThreads, 0, stream>>>(p);
+    else quant_kernel<128, false, false><<<g3, kThreads, 0, stream>>>(p);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || l.tiles_k == 0) return e;
   dim3 g4(l.tiles_k, p.Hkv, p.B);
-  if (p.D == 64) quant_kernel<64, true><<<g4, kThreads, 0, stream>>>(p);
-  else quant_kernel<128, true><<<g4, kThreads, 0, stream>>>(p);
+  if (gs) {
+    if (p.D == 64) quant_kernel<64, true, true><<<g4, kThreads, 0, stream>>>(p);
+    else quant_kernel<128, true, true><<<g4, kThreads, 0, stream>>>(p);
+  } else {
+    if (p.D == 64) quant_kernel<64, true, false><<<g4, kThreads, 0, stream>>>(p);
+    else quant_kernel<128, true, false><<<g4, kThreads, 0, stream>>>(p);
+  }
   return cudaGetLastError();
 }
 

@@ -9,6 +9,10 @@
  * binary32 x, fp32(double(x) * RN64(1/2688)) equals the IEEE binary32 quotient x / 2688
  * (the exact quotient's binary fraction repeats with period 6 -- 2688 = 21 * 2^7 -- so it
  * is never within 2^-52 of a binary32 rounding midpoint; subnormal quotients included).
+ * And the per-element divisions of the quantizers by an arbitrary binary32 divisor d:
+ * fp32(double(x) * c) equals x / d, with c the kernel's double reciprocal (the binary32
+ * reciprocal refined by two Newton steps in double FMAs, d < 2^-64 scaled by 2^64), for
+ * 4000 pseudo-random divisors in [2^-130, 2^21) and every (stride * 641)-th binary32 x.
  * Prints the number of mismatches of each part; exit status 0 when all are 0. */
 #include <math.h>
 #include <stdint.h>
@@ -22,6 +26,16 @@ static uint32_t u_of(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
 static double e4m3_value(int b) {
   const int e = (b >> 3) & 15, m = b & 7;
   return e == 0 ? ldexp(m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+}
+
+static double recip_d(float d) {
+  const int tiny = d < 5.421010862427522e-20f;
+  const float ds = tiny ? d * 18446744073709551616.0f : d;
+  const double dd = (double)ds;
+  double y = (double)(1.0f / ds);
+  y = fma(y, fma(-dd, y, 1.0), y);
+  y = fma(y, fma(-dd, y, 1.0), y);
+  return tiny ? y * 18446744073709551616.0 : y;
 }
 
 static float div_fma(float x, float d, float r) {
@@ -63,7 +77,22 @@ int main(int argc, char** argv) {
     ++n2688;
     if (u_of(ref) != u_of(got)) ++bad2688;
   }
+  long nd = 0, badd = 0;
+  uint32_t lcg = 12345u;
+  for (int gi = 0; gi < 4000; ++gi) {  /* arbitrary divisors: quantizer x / g and x / s */
+    lcg = lcg * 1664525u + 1013904223u;
+    const float d = f_of(0x00000001u + (lcg >> 4) % 0x4A000000u);
+    const double c = recip_d(d);
+    for (uint32_t u = (lcg & 1023u); u < 0x7F800000u; u += stride * 641u) {
+      const float x = f_of(u);
+      volatile float ref = x / d;
+      const float got = (float)((double)x * c);
+      ++nd;
+      if (u_of(ref) != u_of(got)) ++badd;
+    }
+  }
   printf("e4m3 divisors: %ld checks, %ld mismatches; d = 6: %ld checks, %ld mismatches; "
-         "x / 2688 by a double product: %ld checks, %ld mismatches\n", n, bad, n6, bad6, n2688, bad2688);
-  return (bad == 0 && bad6 == 0 && bad2688 == 0) ? 0 : 1;
+         "x / 2688 by a double product: %ld checks, %ld mismatches; x / d by a double product: "
+         "%ld checks, %ld mismatches\n", n, bad, n6, bad6, n2688, bad2688, nd, badd);
+  return (bad == 0 && bad6 == 0 && bad2688 == 0 && badd == 0) ? 0 : 1;
 }
