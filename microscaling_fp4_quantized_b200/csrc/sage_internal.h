@@ -78,7 +78,8 @@ __device__ __forceinline__ bool seq_table_bad(const SeqMap& m) {
 // the division's subroutine out of the attention kernel (measured 1053 -> 1082 TFLOP/s for
 // its general instance on the long workload).
 __device__ __forceinline__ float second_level_scale(float amax) {
-  const float g = __double2float_rn(static_cast<double>(amax) * (1.0 / 2688.0));
+  constexpr double kInvTarget = 1.0 / static_cast<double>(kTwoLevelTarget);
+  const float g = __double2float_rn(static_cast<double>(amax) * kInvTarget);
   return g > 0.0f ? g : 1.0f;
 }
 
