@@ -10,11 +10,14 @@
 //   O  = O * alpha + s1 * P8 V8^T  tcgen05 kind::f8f6f4 (E4M3 x E4M3 -> FP32)
 //   out = diag(s_v) O / l         s_v the channel scales of V
 //
-// Same pipeline as the FP4 kernel (attn_fp4_fwd.cu): warp 0 copies Q once and K / V^T
-// tiles into a 3-stage ring (TMA, 128-byte swizzle), warp 1 allocates TMEM and issues the
-// MMAs (S double-buffered), warps 2-9 are two softmax warpgroups splitting each row's
-// keys; every wait is bounded. 8-bit operands are twice the bytes of FP4 and carry no
-// block scales, so there are no scale-factor copies and no per-16 scale computation.
+// Warp roles: warp 0 copies Q once and K / V^T tiles into a 3-stage ring (TMA, 128-byte
+// swizzle), warp 1 allocates TMEM and issues the MMAs (S double-buffered), warps 2-9 are
+// two softmax warpgroups splitting each row's keys (they exchange the row maxima every
+// tile and each folds half of O). Every wait is bounded. This is the FP4 kernel's earlier
+// design: the FP4 kernel's alternating-warpgroup design measured slower for these 8-bit
+// products, which take twice the tensor time and twice the SMEM bytes of FP4. 8-bit
+// operands carry no block scales, so there are no scale-factor copies and no per-16
+// scale computation.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
