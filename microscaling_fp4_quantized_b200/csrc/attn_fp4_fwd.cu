@@ -26,6 +26,9 @@ cudaError_t launch_attention(const TensorMaps& m, const AttnParams& p, int tiles
   const bool general = p.seq.cu_q != nullptr || p.seq.Nq != p.seq.Nk || p.amax != nullptr;
   const int mode = p.qk_bias != nullptr ? 2 : (general ? 1 : 0);
   if (p.causal) return launch_attention_causal(m, p, tiles_q, mode, stream);
+  // Few query tiles per (sequence, head): the persistent form hides each CTA's start-up
+  // (measured at D = 128: 805 against 727 TFLOP/s on B64 H32 N1024; long rows unchanged).
+  if (mode == 0 && p.D == 128 && tiles_q <= kShortTiles) return launch_attention_short(m, p, tiles_q, stream);
   return p.D == 64 ? launch_attn_full_d<64>(m, p, tiles_q, mode, stream)
                    : launch_attn_full_d<128>(m, p, tiles_q, mode, stream);
 }

@@ -158,6 +158,7 @@ struct AttnParams {
   uint32_t* err;        // device error word
   uint64_t timeout_ns;  // bound on every wait
   uint32_t debug_flags; // kDebugNoLoads: the producer issues no copies (test of the error path)
+  int tiles_q;          // query tiles of the longest sequence (set by the persistent launcher)
 };
 
 enum : uint32_t { kDebugNoLoads = 1u };
@@ -175,5 +176,9 @@ cudaError_t launch_quantize8(const QuantParams& p, const QuantLaunch& l, cudaStr
 cudaError_t launch_attention(const TensorMaps& maps, const AttnParams& p, int tiles_q, cudaStream_t stream);
 cudaError_t launch_qk_scores(const TensorMaps& maps, const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_attention8(const TensorMaps& maps, const AttnParams& p, int tiles_q, cudaStream_t stream);
+// The persistent FP4 attention kernel (square dense, one-level scales, non-causal), used
+// by launch_attention at D = 128 when there are at most kShortTiles query tiles.
+cudaError_t launch_attention_short(const TensorMaps& maps, const AttnParams& p, int tiles_q, cudaStream_t stream);
+constexpr int kShortTiles = 8;
 
 }  // namespace sage
