@@ -85,6 +85,11 @@ constexpr uint32_t kColSfQ = 384;   // 4 columns per 64-wide K chunk of D
 constexpr uint32_t kColSfK = 392;   // + 8 * K stage
 constexpr uint32_t kColSfV = 424;   // + 8 * V stage
 constexpr uint32_t kColSfP = 456;   // + 8 * P buffer (ends at 472)
+// The TMEM regions must not overlap (S buffers, PV, then the scale-factor columns).
+static_assert(kColPV >= kColS0 + 2 * 128 && kColSfQ >= kColPV + 128, "TMEM: S / PV regions");
+static_assert(kColSfK >= kColSfQ + 8 && kColSfV >= kColSfK + 8 * kKStages &&
+                  kColSfP >= kColSfV + 8 * kVStages && kColSfP + 16 <= kTmemCols,
+              "TMEM: scale-factor columns");
 
 template <int D, bool QB = false>
 struct Layout {

@@ -49,6 +49,11 @@ constexpr uint32_t kColSfQ = 384;   // + 8 * Q slot; 4 columns per 64-wide K chu
 constexpr uint32_t kColSfK = 400;   // + 8 * K stage
 constexpr uint32_t kColSfV = 432;   // + 8 * V stage
 constexpr uint32_t kColSfP = 464;   // + 8 * P buffer (ends at 480)
+// The TMEM regions must not overlap (S buffers, PV, then the scale-factor columns).
+static_assert(kColPV >= kColS0 + 2 * 128 && kColSfQ >= kColPV + 128, "TMEM: S / PV regions");
+static_assert(kColSfK >= kColSfQ + 16 && kColSfV >= kColSfK + 8 * kKStages &&
+                  kColSfP >= kColSfV + 8 * kVStages && kColSfP + 16 <= kTmemCols,
+              "TMEM: scale-factor columns");
 
 template <int D, bool QB = false>
 struct Layout {
