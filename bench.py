@@ -35,6 +35,22 @@ FP4_NOMINAL_TFLOPS = 9000.0
 FP4_PER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
 
 
+def fp4_peak(peaks: dict, basis: str, probe=None, b8: bool = False):
+    """Roofline denominator of the attention kernel (timed per launch, in isolation: the
+    burst figure). FP4: the measured bf16 burst rate x 4 (nominal FP4 : BF16), or the
+    measured rate of the FP4 instruction itself (sage.mma_rate) when that is higher;
+    8-bit: bf16 burst x 2. Returns (TFLOP/s, description)."""
+    burst = peaks.get("bf16_tflops", peaks.get("bf16_tflops_sustained"))
+    ratio = 2.0 if b8 else FP4_PER_BF16
+    peak = ratio * burst
+    how = f"{basis} bf16 burst {burst} TFLOP/s x {ratio:g} (nominal {'8-bit' if b8 else 'FP4'}:BF16)"
+    if probe is not None and not b8 and probe["tflops"] > peak:
+        peak = probe["tflops"]
+        how = (f"measured FP4 tensor-core rate (tcgen05 mxf4nvf4 M128 N{probe['n']} K64, "
+               f"{probe['ctas']} CTAs), above the bf16-derived {ratio * burst:.0f}")
+    return peak, how
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -125,6 +141,58 @@ def _attn_traffic(wl, b8=False):
     # attention traffic is the quantized inputs plus the output: it scales with B*H*N
     scale = (wl.B * wl.H * wl.N) / (cap.B * cap.H * cap.N)
     return float(rec["dram_bytes_per_launch"]) * scale, f"ncu capture of {cap.name}, scaled by B*H*N"
+
+
+TRAFFIC_SOURCES = {
+    False: ("attn_fp4_fwd_kernel", "attn_fp4_fwd_kernel_traffic.json",
+            ["microscaling_fp4_quantized_b200/csrc/attn_fp4_kernel.cuh",
+             "microscaling_fp4_quantized_b200/csrc/attn_common.cuh",
+             "microscaling_fp4_quantized_b200/csrc/sm100_ptx.cuh",
+             "microscaling_fp4_quantized_b200/csrc/sage_internal.h"]),
+    True: ("attn8_fwd_kernel", "attn8_fwd_kernel_traffic.json",
+           ["microscaling_fp4_quantized_b200/csrc/attn8_fwd.cu",
+            "microscaling_fp4_quantized_b200/csrc/attn_common.cuh",
+            "microscaling_fp4_quantized_b200/csrc/sm100_ptx.cuh",
+            "microscaling_fp4_quantized_b200/csrc/sage_internal.h"]),
+}
+
+_BYTE_UNITS = {"byte": 1.0, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9, "tbyte": 1e12,
+               "kibyte": 1024.0, "mibyte": 1024.0 ** 2, "gibyte": 1024.0 ** 3}
+
+
+def write_traffic_record(csv_path: str, wl, b8: bool) -> dict:
+    """Traffic record of the attention kernel from an ncu CSV of one launch
+    (--metrics dram__bytes_read.sum,dram__bytes_write.sum --csv), hashed over the kernel's
+    sources as they are now: run it right after the capture, on the same tree."""
+    import csv
+    import hashlib
+    kernel, name, sources = TRAFFIC_SOURCES[b8]
+    total, launches = {}, set()
+    with open(csv_path, newline="") as f:
+        rows = [r for r in csv.reader(f)]
+    head = next(i for i, r in enumerate(rows) if "Metric Name" in r)
+    cols = rows[head]
+    ki, mi, ui, vi, ii = (cols.index(c) for c in ("Kernel Name", "Metric Name", "Metric Unit", "Metric Value", "ID"))
+    for r in rows[head + 1:]:
+        if len(r) <= vi or kernel not in r[ki] or r[mi] not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            continue
+        launches.add(r[ii])
+        total[r[ii]] = total.get(r[ii], 0.0) + float(r[vi].replace(",", "")) * _BYTE_UNITS[r[ui].strip().lower()]
+    if not total:
+        raise RuntimeError(f"no {kernel} DRAM metrics in {csv_path}")
+    h = hashlib.sha256()
+    for src in sources:
+        with open(os.path.join(ROOT, src), "rb") as f:
+            h.update(f.read())
+    rec = {"kernel": kernel, "sources": sources, "source_sha256_prefix": h.hexdigest()[:16],
+           "captured_workload": wl.name, "launches_captured": len(launches),
+           "dram_bytes_per_launch": statistics.mean(total.values()),
+           "note": "dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture (per launch); "
+                   "written by bench.py --write-traffic from that capture's CSV; reported only while the "
+                   "hash of the sources matches"}
+    with open(os.path.join(ROOT, "profiles", name), "w") as f:
+        json.dump(rec, f, indent=1)
+    return rec
 
 
 def max_over_ranks(value: float, dist, device) -> float:
@@ -220,7 +288,9 @@ def run_sweep(args):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     peaks, basis = _peaks()
-    fp4_peak = FP4_PER_BF16 * peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    probe = sage.mma_rate(n=128)
+    peak_tflops, peak_how = fp4_peak(peaks, basis, probe)
+    print(json.dumps({"fp4_mma_probe": probe, "peak_tflops": peak_tflops, "peak_basis": peak_how}), flush=True)
     for wl in [workloads.TINY, workloads.MEDIUM, workloads.LLM_CAUSAL, workloads.LONG] + workloads.SWEEP:
         q, k, v = workloads.make_inputs(wl)
         qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
@@ -262,8 +332,9 @@ def run_sweep(args):
         print(json.dumps({
             "workload": wl.name, "ops": wl.ops, "tops": wl.ops / (ms * 1e-3) / 1e12, "ms": ms,
             "attn_tops": wl.ops / (ms_attn * 1e-3) / 1e12, "attn_ms": ms_attn,
-            "pct_of_fp4_peak": 100.0 * wl.ops / (ms * 1e-3) / 1e12 / fp4_peak,
-            "peak_basis": f"{basis} bf16 sustained x {FP4_PER_BF16:g}",
+            "pct_of_fp4_peak": 100.0 * wl.ops / (ms * 1e-3) / 1e12 / peak_tflops,
+            "attn_pct_of_fp4_peak": 100.0 * wl.ops / (ms_attn * 1e-3) / 1e12 / peak_tflops,
+            "pct_of_nominal_fp4": 100.0 * wl.ops / (ms * 1e-3) / 1e12 / FP4_NOMINAL_TFLOPS,
             "vs_emulated": {"cos": m_em["cos"], "max_abs_over_max_v": m_em["max_abs"] / float(np.abs(vh).max())},
             "vs_exact": {"cos": m_ex["cos"], "rel_l1": m_ex["rel_l1"], "rmse": m_ex["rmse"]},
             "sampled_rows": int(len(rows)), "device_error_word": err,
@@ -415,7 +486,16 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="measure every named configuration (one JSON line each) instead of "
                          "the single bench line")
+    ap.add_argument("--write-traffic", metavar="CSV",
+                    help="write the attention kernel's traffic record under profiles/ from the CSV of "
+                         "an ncu capture of this workload and exit")
+    ap.add_argument("--no-mma-probe", action="store_true",
+                    help="skip the FP4 tensor-core rate probe that sets the roofline peak")
     args = ap.parse_args()
+    if args.write_traffic:
+        print(json.dumps(write_traffic_record(args.write_traffic, workloads.by_name(args.workload),
+                                              args.precision == "8bit")))
+        return 0
     if args.sweep:
         return run_sweep(args)
     wl = workloads.by_name(args.workload)
@@ -449,6 +529,10 @@ def main():
         plan.attention(out)
         if ev_end is not None:
             ev_end.record(stream)
+
+    probe = None
+    if not args.no_mma_probe and args.precision == "fp4":
+        probe = sage.mma_rate(n=128)       # the FP4 instruction's own measured rate
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -516,22 +600,18 @@ def main():
         return 0
 
     peaks, basis = _peaks()
-    sustained = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
-    fp4_peak = FP4_PER_BF16 * sustained
+    b8 = args.precision == "8bit"
+    peak, peak_how = fp4_peak(peaks, basis, probe, b8)
     attn_avg_ms = statistics.mean(attn_ms)
     achieved = wl.ops / (attn_avg_ms * 1e-3) / 1e12
-    b8 = args.precision == "8bit"
     traffic, traffic_src = _attn_traffic(wl, b8)
-    if b8:
-        # FP8 / INT8 tensor peak: measured bf16 x 2 (nominal 8-bit : BF16 = 4.5 : 2.25)
-        fp4_peak = 2.0 * sustained
+    nominal = FP4_NOMINAL_TFLOPS / 2 if b8 else FP4_NOMINAL_TFLOPS
     roofline = {
         "kernel": "attn8_fwd_kernel" if b8 else "attn_fp4_fwd_kernel", "bound": "tensor", "achieved": achieved,
-        "peak": fp4_peak,
-        "unit": "TFLOP/s", "frac": achieved / fp4_peak, "traffic": traffic, "traffic_source": traffic_src,
-        "peak_basis": (f"{basis} bf16 sustained {sustained} TFLOP/s x 2 (nominal 8-bit:BF16)" if b8 else
-                       f"{basis} bf16 sustained {sustained} TFLOP/s x {FP4_PER_BF16:g} (nominal FP4:BF16)"),
-        "frac_of_nominal": achieved / (FP4_NOMINAL_TFLOPS / 2 if b8 else FP4_NOMINAL_TFLOPS),
+        "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+        "traffic_source": traffic_src, "peak_basis": peak_how,
+        "frac_of_nominal": achieved / nominal, "nominal_tflops": nominal,
+        "fp4_mma_probe_tflops": None if probe is None else probe["tflops"],
         "attn_ms": attn_avg_ms, "quant_ms": statistics.mean(quant_ms),
     }
     cpu = None
@@ -548,7 +628,8 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": "int8_e4m3" if b8 else "fp4_e2m1", "data": "synthetic",
         "config": cfg, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clocks, "device_error_word": err,
-        "pct_of_fp4_peak": 100.0 * value / world / fp4_peak,
+        "pct_of_fp4_peak": 100.0 * value / world / peak,
+        "pct_of_nominal_fp4": 100.0 * value / world / nominal,
     }
     if variants is not None:
         line["variants"] = variants

@@ -262,7 +262,10 @@ sage_status_t sage_fp4_attn_fwd(const void* q, const void* k, const void* v, voi
  *     B*H = 16, N = 4096, D = 128); larger problems return SAGE_ERR_UNSUPPORTED before
  *     anything is launched.
  *   - The first call on a device looks up the array's device address (with that device
- *     current) and caches it; make that first call before any stream capture.
+ *     current) and caches it; make that first call before any stream capture. The cache
+ *     lives as long as the process: do not use this entry point on a device after
+ *     cudaDeviceReset() or any other teardown of its primary context (the cached address
+ *     would belong to the destroyed context).
  *   - Every call shares the one array, which keeps the last call's contents. Nothing in
  *     it has to start at zero (each call writes every byte it later reads), but calls
  *     that overlap on the GPU (different streams, or different host threads, on the same
@@ -303,6 +306,19 @@ const char* sage_fp4_last_cuda_error(void);
  * rejected with SAGE_ERR_INVALID_ARG.
  */
 sage_status_t sage_fp4_set_debug_flags(uint32_t flags);
+
+/*
+ * Rate probe of the FP4 tensor cores the method runs on (SageAttention3 abstract, "FP4
+ * Tensor Cores in Blackwell GPUs"): the block-scaled FP4 instruction both attention
+ * contractions use (tcgen05.mma kind::mxf4nvf4, block 16, E2M1 operands, UE4M3 scales,
+ * M = 128, N = n, K = 64). Launches `ctas` CTAs of one per SM; each issues `iters`
+ * products back to back from operands resident in its shared memory and waits (bounded)
+ * for them. The caller times the launch (for instance with CUDA events on `stream`);
+ * it performs 2 * 128 * n * 64 * iters * ctas operations. n must be 64 or 128, iters and
+ * ctas positive (ctas <= 65535), else SAGE_ERR_INVALID_ARG. Reads and writes no caller
+ * memory; the products themselves are discarded.
+ */
+sage_status_t sage_fp4_mma_rate(int n, int iters, int ctas, void* stream);
 
 /*
  * Bound on every in-kernel wait, in nanoseconds (default 2e9; 0 restores the default).

@@ -37,7 +37,7 @@ EXPORTED = [
     "sage_fp4_attn_fwd_ex", "sage_fp4_attn_fwd", "sage_fp4_qk_scores",
     "sage_fp4_get_device_error", "sage_fp4_set_wait_timeout_ns", "sage_fp4_attn_fwd_noalloc",
     "sage_fp4_last_cuda_error", "sage_fp4_set_debug_flags", "sage_fp4_problem_sizes",
-    "sage_fp4_quantize", "sage_fp4_attn_quantized", "sage_fp4_attn",
+    "sage_fp4_quantize", "sage_fp4_attn_quantized", "sage_fp4_attn", "sage_fp4_mma_rate",
 ]
 
 
@@ -119,6 +119,7 @@ def lib():
         L.sage_fp4_quantize.argtypes = [pp, vp, vp, vp, ctypes.POINTER(_Quantized), vp, sz, vp]
         L.sage_fp4_attn_quantized.argtypes = [pp, ctypes.POINTER(_Quantized), vp, vp]
         L.sage_fp4_attn.argtypes = [pp, vp, vp, vp, vp, vp, sz, vp]
+        L.sage_fp4_mma_rate.argtypes = [i, i, i, vp]
         for n in EXPORTED[1:]:
             if n not in ("sage_fp4_quantize_scratch_bytes", "sage_fp4_workspace_bytes",
                          "sage_fp4_last_cuda_error"):
@@ -290,6 +291,31 @@ def set_debug_flags(flags: int) -> None:
     """Test switch: bit 0 makes the attention kernel issue no loads, so its bounded waits
     run out and the device error word reports a timeout (0 restores normal operation)."""
     _check(lib().sage_fp4_set_debug_flags(int(flags)), "sage_fp4_set_debug_flags")
+
+
+def mma_rate(n: int = 128, iters: int = 200000, ctas: Optional[int] = None, repeats: int = 5,
+             device=None) -> dict:
+    """Measured rate of the block-scaled FP4 tensor-core instruction (M128 x N x K64) with
+    one CTA per SM: the best of `repeats` CUDA-event timings of sage_fp4_mma_rate after one
+    warm-up launch. Returns {"tflops", "ms", "ops", "ctas", "n"}."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    if ctas is None:
+        ctas = torch.cuda.get_device_properties(dev).multi_processor_count
+    s = _stream(dev)
+    _check(lib().sage_fp4_mma_rate(n, max(1, iters // 10), ctas, s), "sage_fp4_mma_rate")
+    best = None
+    for _ in range(repeats):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        _check(lib().sage_fp4_mma_rate(n, iters, ctas, s), "sage_fp4_mma_rate")
+        b.record()
+        torch.cuda.synchronize(dev)
+        ms = a.elapsed_time(b)
+        best = ms if best is None else min(best, ms)
+    if device_error(dev) != 0:
+        raise SageError(SAGE_ERR_TIMEOUT, "sage_fp4_mma_rate")
+    ops = 2.0 * 128 * n * 64 * iters * ctas
+    return {"tflops": ops / best / 1e9, "ms": best, "ops": ops, "ctas": ctas, "n": n}
 
 
 def default_sm_scale(D: int) -> float:

@@ -632,6 +632,13 @@ sage_status_t sage_fp4_set_debug_flags(uint32_t flags) {
   return SAGE_OK;
 }
 
+sage_status_t sage_fp4_mma_rate(int n, int iters, int ctas, void* stream) {
+  if ((n != 64 && n != 128) || iters < 1 || ctas < 1 || ctas > 65535) return SAGE_ERR_INVALID_ARG;
+  uint32_t* err = nullptr;
+  if (sage_status_t st = error_word(&err); st != SAGE_OK) return st;
+  return cuda_status(sage::launch_mma_rate(n, iters, ctas, err, g_timeout_ns.load(), static_cast<cudaStream_t>(stream)));
+}
+
 sage_status_t sage_fp4_set_wait_timeout_ns(uint64_t ns) {
   g_timeout_ns.store(ns == 0 ? kDefaultTimeoutNs : ns);
   return SAGE_OK;

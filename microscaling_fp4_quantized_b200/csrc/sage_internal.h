@@ -180,5 +180,8 @@ cudaError_t launch_attention8(const TensorMaps& maps, const AttnParams& p, int t
 // by launch_attention at D = 128 when there are at most kShortTiles query tiles.
 cudaError_t launch_attention_short(const TensorMaps& maps, const AttnParams& p, int tiles_q, cudaStream_t stream);
 constexpr int kShortTiles = 8;
+// Tensor-core rate probe (mma_rate.cu): `ctas` CTAs, each issuing `iters` block-scaled FP4
+// products of M = 128, N = n, K = 64.
+cudaError_t launch_mma_rate(int n, int iters, int ctas, uint32_t* err, uint64_t timeout_ns, cudaStream_t stream);
 
 }  // namespace sage

@@ -26,7 +26,10 @@ void* g_scratch_addr[kMaxDevices] = {};
 std::mutex g_scratch_mu;
 
 // Device address of the array on the current device. Host code must not use the
-// symbol itself: on the host it names a stand-in object, not device memory.
+// symbol itself: on the host it names a stand-in object, not device memory. The address
+// is cached per device for the life of the process, so it is only valid while the
+// device's primary context lives: the library must not be used on a device after a
+// cudaDeviceReset() or another teardown of that context.
 sage_status_t scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SAGE_ERR_CUDA;

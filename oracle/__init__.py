@@ -65,6 +65,7 @@ def _L():
             "so_attn_emulated": [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, c_long, c_long, c_long,
                                  c_long, c_long, c_long, c_int, c_double, c_long, vp, c_long, vp],
             "so_qk_bias": [vp, vp, vp, c_long, c_long, c_long, c_long, c_long, vp],
+            "so_attn_from_scores": [vp, c_long, c_long, vp, vp, vp, vp, vp, c_long, c_long, vp],
             "so_quant_int8_rows": [vp, c_long, c_long, c_long, c_long, vp, vp, vp],
             "so_quant_e4m3_channels": [vp, c_long, c_long, c_long, vp, vp],
             "so_attn_emulated8": [vp, vp, vp, vp, vp, vp, c_long, c_long, c_long, c_long, c_long,
@@ -286,6 +287,27 @@ def attn_emulated(qz: dict, causal: bool, sm_scale: float, Bk: int = 128, rows=N
     return out.reshape(B * Hq, Nq, D) if rows is None else out
 
 
+def attn_from_scores(S, kv, n_keys, qz: dict, Bk: int = 128) -> np.ndarray:
+    """The emulated attention's softmax, two-level P~ quantization and P^ V~ accumulation
+    applied to GIVEN scores: S [n_rows, Nk] (already multiplied by sm_scale, and by the Q
+    and K second-level scales when there are any), row r reading the values of key/value
+    head kv[r] of qz (the output of quantize_qkv) and seeing keys 0 .. n_keys[r] - 1.
+    Returns [n_rows, D] binary64. Used to check a GPU row against the method applied to
+    that GPU's own FP32 scores."""
+    S = np.ascontiguousarray(np.asarray(S, np.float64))
+    n_rows, Nk = S.shape
+    assert Nk == qz["Nk"]
+    kv = np.ascontiguousarray(np.asarray(kv, np.int64).reshape(n_rows))
+    nk = np.ascontiguousarray(np.asarray(n_keys, np.int64).reshape(n_rows))
+    D = qz["D"]
+    out = np.empty((n_rows, D), np.float64)
+    vt, vsf = np.ascontiguousarray(qz["vt_codes"]), np.ascontiguousarray(qz["vt_sf"])
+    gv = None if qz["gv"] is None else _f32(qz["gv"])
+    _L().so_attn_from_scores(_p(S), n_rows, Nk, _p(kv), _p(nk), _p(vt), _p(vsf),
+                             _p(gv) if gv is not None else None, D, int(Bk), _p(out))
+    return out
+
+
 def attn_exact(q, k, v, causal: bool, sm_scale: float, rows=None, heads=None) -> np.ndarray:
     """Two-pass softmax attention in binary64 -> [n_rows, D] (or [B*Hq, Nq, D]).
     q [B*Hq, Nq, D]; k, v [B*Hkv, Nk, D]; heads = (B, Hq, Hkv) as in quantize_qkv."""
@@ -482,14 +504,24 @@ def attention8(q, k, v, causal: bool, sm_scale: float, Bk: int = 128, rows=None,
 
 def metrics(x: np.ndarray, ref: np.ndarray) -> dict:
     """Cosine similarity, relative L1 and RMSE (the accuracy metrics the SageAttention
-    thread reports): cos = sum(xy)/sqrt(sum x^2 sum y^2), relL1 = sum|x-y|/sum|y|,
-    rmse = sqrt(mean((x-y)^2)); plus max |x - y|."""
-    x = np.asarray(x, np.float64).ravel()
-    y = np.asarray(ref, np.float64).ravel()
-    den = np.sqrt((x * x).sum() * (y * y).sum())
+    thread reports, reply to reviewer tyTT W1): cos = sum(xy)/sqrt(sum x^2 sum y^2),
+    relL1 = sum|x-y|/sum|y|, rmse = sqrt(mean((x-y)^2)); plus max |x - y| over every
+    element. x and ref must have the same shape. cos is 1 when both are all zeros and 0
+    when exactly one of them is (an all-zero output never passes as similar)."""
+    x = np.asarray(x, np.float64)
+    y = np.asarray(ref, np.float64)
+    if x.shape != y.shape:
+        raise ValueError(f"metrics: shapes differ {x.shape} vs {y.shape}")
+    x, y = x.ravel(), y.ravel()
+    nx, ny = (x * x).sum(), (y * y).sum()
+    if nx > 0 and ny > 0:
+        cos = float((x * y).sum() / np.sqrt(nx * ny))
+    else:
+        cos = 1.0 if nx == 0 and ny == 0 else 0.0
+    sy = np.abs(y).sum()
     return {
-        "cos": float((x * y).sum() / den) if den > 0 else 1.0,
-        "rel_l1": float(np.abs(x - y).sum() / max(np.abs(y).sum(), 1e-300)),
-        "rmse": float(np.sqrt(np.mean((x - y) ** 2))),
+        "cos": cos,
+        "rel_l1": float(np.abs(x - y).sum() / sy) if sy > 0 else (0.0 if not np.abs(x).any() else float("inf")),
+        "rmse": float(np.sqrt(np.mean((x - y) ** 2))) if x.size else 0.0,
         "max_abs": float(np.abs(x - y).max()) if x.size else 0.0,
     }

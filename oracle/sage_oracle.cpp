@@ -290,6 +290,70 @@ void so_qk_bias(const float* mu_q, const float* k, const float* mu_k, long B, lo
   }
 }
 
+}  // extern "C"
+
+namespace {
+
+// The key-tile walk of one query row (steps of so_attn_emulated below): S[0..n_keys) are
+// the row's scaled scores (binary64), keys at or past n_keys are masked; vd [>= n_keys, D]
+// the dequantized values. Writes O / l (0 for a row that sees no key) to out[0..D).
+void walk_key_tiles(const double* S, long n_keys, const double* vd, long D, long Bk, double* out) {
+  std::vector<double> O(static_cast<size_t>(D), 0.0), P(static_cast<size_t>(Bk));
+  std::vector<float> P2(static_cast<size_t>(Bk + 16));
+  std::vector<double> phat(static_cast<size_t>(Bk + 16));
+  double m = -std::numeric_limits<double>::infinity(), l = 0.0;
+  for (long j0 = 0; j0 < n_keys; j0 += Bk) {
+    const long j1 = std::min(j0 + Bk, n_keys);  // exclusive; keys past it are masked
+    double tmax = -std::numeric_limits<double>::infinity();
+    for (long j = j0; j < j1; ++j) tmax = std::max(tmax, S[j]);
+    const double m_new = std::max(m, tmax);
+    const double alpha = std::exp(m - m_new);  // exp(-inf) = 0 on the first tile
+    double rowsum = 0.0, r = 0.0;
+    for (long j = j0; j < j1; ++j) {
+      P[j - j0] = std::exp(S[j] - m_new);
+      rowsum += P[j - j0];
+      r = std::max(r, P[j - j0]);
+    }
+    l = l * alpha + rowsum;
+    const double s1 = r / kTwoLevelTarget;
+    // P2 over the whole tile width (masked or absent keys are 0), blocks of 16.
+    const long width = std::min(Bk, ((j1 - j0) + 15) / 16 * 16);
+    for (long t = 0; t < width; ++t)
+      P2[t] = (j0 + t < j1) ? static_cast<float>(P[t] / s1) : 0.0f;
+    for (long b0 = 0; b0 < width; b0 += 16) {
+      uint8_t codes[16], sb;
+      quant_block16(&P2[b0], 1, 16, codes, &sb);
+      const double s = e4m3_value(sb);
+      for (int t = 0; t < 16; ++t) phat[b0 + t] = e2m1_value(codes[t]) * s;
+    }
+    for (long d = 0; d < D; ++d) {
+      double acc = 0.0;
+      for (long j = j0; j < j1; ++j) acc += phat[j - j0] * vd[j * D + d];
+      O[d] = O[d] * alpha + s1 * acc;
+    }
+    m = m_new;
+  }
+  for (long d = 0; d < D; ++d) out[d] = l > 0.0 ? O[d] / l : 0.0;
+}
+
+// Dequantized V~ [Nk, D] of key/value head kv (binary64, exact): e2m1(code) * s * g_v.
+void dequant_v(const uint8_t* vt_codes, const uint8_t* vt_sf, long kv, long Nk, long D, double g_v,
+               std::vector<double>& vd) {
+  const long Nkp = (Nk + 15) / 16 * 16, nb_n = Nkp / 16;
+  vd.assign(static_cast<size_t>(Nk * D), 0.0);
+#pragma omp parallel for schedule(static)
+  for (long n = 0; n < Nk; ++n)
+    for (long d = 0; d < D; ++d) {
+      const uint8_t* vr = vt_codes + (kv * D + d) * (Nkp / 2);
+      const double sv = e4m3_value(vt_sf[(kv * D + d) * nb_n + n / 16]);
+      vd[n * D + d] = e2m1_value(get_nibble(vr, n)) * sv * g_v;
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
 // ------------------------------------------------------ emulated attention ----
 // One or more sequences of equal lengths: B batches, Hq query heads, Hkv key/value heads
 // (query head h reads key/value head h / (Hq / Hkv)), Nq queries and Nk keys each.
@@ -315,8 +379,7 @@ void so_attn_emulated(const uint8_t* q_codes, const uint8_t* q_sf, const uint8_t
                       double sm_scale, long Bk, const long* rows, long n_rows, double* out) {
   (void)B;
   const long group = Hq / Hkv;
-  const long Nkp = (Nk + 15) / 16 * 16;
-  const long nb_d = D / 16, nb_n = Nkp / 16;
+  const long nb_d = D / 16;
   // Group rows by key/value head so that K~ and V~ are dequantized once per head.
   auto kv_of = [&](long bhq) { return (bhq / Hq) * Hkv + (bhq % Hq) / group; };
   std::vector<long> order(static_cast<size_t>(n_rows));
@@ -333,74 +396,53 @@ void so_attn_emulated(const uint8_t* q_codes, const uint8_t* q_sf, const uint8_t
     const double g_k = gk ? gk[kv] : 1.0, g_v = gv ? gv[kv] : 1.0;
 
     kd.assign(static_cast<size_t>(Nk * D), 0.0);
-    vd.assign(static_cast<size_t>(Nk * D), 0.0);
 #pragma omp parallel for schedule(static)
     for (long n = 0; n < Nk; ++n) {
       const uint8_t* kr = k_codes + (kv * Nk + n) * (D / 2);
       for (long d = 0; d < D; ++d) {
         const double s = e4m3_value(k_sf[(kv * Nk + n) * nb_d + d / 16]);
         kd[n * D + d] = e2m1_value(get_nibble(kr, d)) * s * g_k;
-        const uint8_t* vr = vt_codes + (kv * D + d) * (Nkp / 2);
-        const double sv = e4m3_value(vt_sf[(kv * D + d) * nb_n + n / 16]);
-        vd[n * D + d] = e2m1_value(get_nibble(vr, n)) * sv * g_v;
       }
     }
+    dequant_v(vt_codes, vt_sf, kv, Nk, D, g_v, vd);
 
 #pragma omp parallel for schedule(dynamic, 1)
     for (long rr = r0; rr < r1; ++rr) {
       const long ridx = order[rr];
       const long bhq = rows[2 * ridx], i = rows[2 * ridx + 1];
       const double g_q = gq ? gq[bhq] : 1.0;
-      std::vector<double> qd(static_cast<size_t>(D)), O(static_cast<size_t>(D), 0.0);
-      std::vector<double> S(static_cast<size_t>(Bk)), P(static_cast<size_t>(Bk));
-      std::vector<float> P2(static_cast<size_t>(Bk + 16));
-      std::vector<double> phat(static_cast<size_t>(Bk + 16));
+      std::vector<double> qd(static_cast<size_t>(D));
       const uint8_t* qr = q_codes + (bhq * Nq + i) * (D / 2);
       for (long d = 0; d < D; ++d)
         qd[d] = e2m1_value(get_nibble(qr, d)) * e4m3_value(q_sf[(bhq * Nq + i) * nb_d + d / 16]) * g_q;
-
-      double m = -std::numeric_limits<double>::infinity(), l = 0.0;
+      // Keys j <= last_key are visible; the rest of the row is masked.
       const long last_key = causal ? std::min(i + (Nk - Nq), Nk - 1) : Nk - 1;
-      for (long j0 = 0; j0 <= last_key; j0 += Bk) {
-        const long j1 = std::min(j0 + Bk, last_key + 1);  // exclusive; keys past it are masked
-        double tmax = -std::numeric_limits<double>::infinity();
-        for (long j = j0; j < j1; ++j) {
-          double acc = 0.0;
-          for (long d = 0; d < D; ++d) acc += qd[d] * kd[j * D + d];
-          if (qk_bias) acc += qk_bias[bhq * Nk + j];
-          S[j - j0] = sm_scale * acc;
-          tmax = std::max(tmax, S[j - j0]);
-        }
-        const double m_new = std::max(m, tmax);
-        const double alpha = std::exp(m - m_new);  // exp(-inf) = 0 on the first tile
-        double rowsum = 0.0, r = 0.0;
-        for (long j = j0; j < j1; ++j) {
-          P[j - j0] = std::exp(S[j - j0] - m_new);
-          rowsum += P[j - j0];
-          r = std::max(r, P[j - j0]);
-        }
-        l = l * alpha + rowsum;
-        const double s1 = r / kTwoLevelTarget;
-        // P2 over the whole tile width (masked or absent keys are 0), blocks of 16.
-        const long width = std::min(Bk, ((j1 - j0) + 15) / 16 * 16);
-        for (long t = 0; t < width; ++t)
-          P2[t] = (j0 + t < j1) ? static_cast<float>(P[t] / s1) : 0.0f;
-        for (long b0 = 0; b0 < width; b0 += 16) {
-          uint8_t codes[16], sb;
-          quant_block16(&P2[b0], 1, 16, codes, &sb);
-          const double s = e4m3_value(sb);
-          for (int t = 0; t < 16; ++t) phat[b0 + t] = e2m1_value(codes[t]) * s;
-        }
-        for (long d = 0; d < D; ++d) {
-          double acc = 0.0;
-          for (long j = j0; j < j1; ++j) acc += phat[j - j0] * vd[j * D + d];
-          O[d] = O[d] * alpha + s1 * acc;
-        }
-        m = m_new;
+      const long n_keys = std::max(last_key + 1, 0L);
+      std::vector<double> S(static_cast<size_t>(std::max(n_keys, 1L)));
+      for (long j = 0; j < n_keys; ++j) {
+        double acc = 0.0;
+        for (long d = 0; d < D; ++d) acc += qd[d] * kd[j * D + d];
+        if (qk_bias) acc += qk_bias[bhq * Nk + j];
+        S[j] = sm_scale * acc;
       }
-      for (long d = 0; d < D; ++d) out[ridx * D + d] = l > 0.0 ? O[d] / l : 0.0;
+      walk_key_tiles(S.data(), n_keys, vd.data(), D, Bk, out + ridx * D);
     }
     r0 = r1;
+  }
+}
+
+// Steps 5-6 of so_attn_emulated on GIVEN scores: S [n_rows, Nk] binary64 are the
+// already-scaled scores of each row (for instance a GPU's FP32 products, widened); row r
+// reads values of key/value head kv[r] and sees keys 0 .. n_keys[r] - 1. The online
+// softmax, the two-level P~ quantization and the P^ V~ accumulation are exactly those of
+// so_attn_emulated; only the scores come from outside. out: [n_rows, D].
+void so_attn_from_scores(const double* S, long n_rows, long Nk, const long* kv, const long* n_keys,
+                         const uint8_t* vt_codes, const uint8_t* vt_sf, const float* gv, long D,
+                         long Bk, double* out) {
+  std::vector<double> vd;
+  for (long r = 0; r < n_rows; ++r) {
+    dequant_v(vt_codes, vt_sf, kv[r], Nk, D, gv ? gv[kv[r]] : 1.0, vd);
+    walk_key_tiles(S + r * Nk, std::min(n_keys[r], Nk), vd.data(), D, Bk, out + r * D);
   }
 }
 

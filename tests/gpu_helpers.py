@@ -198,3 +198,29 @@ def canonical8(qz: dict, lens_q, lens_k, Hq: int, Hkv: int, D: int) -> list:
         o["k_mean"] = kmean[b * Hkv * D:(b + 1) * Hkv * D].reshape(Hkv, D)
         res.append(o)
     return res
+
+
+def gpu_row_scores(sage, qz: dict, lens_q, lens_k, Hq: int, Hkv: int, D: int, b: int, h: int) -> np.ndarray:
+    """The GPU tensor core's own FP32 products Q^ K^^T (no scale) of query head h of
+    sequence b of a general problem, from the quantized buffers of sage.quantize:
+    [Lq, Lk] float64. The (sequence, head) blocks of Q and of key/value head h / (Hq/Hkv)
+    are copied into a dense one-head problem padded to a common length, and the
+    library's scores kernel (the attention kernel's MMA form) runs on it."""
+    pq, pk = padded_offsets(lens_q), padded_offsets(lens_k)
+    Lq, Lk = int(lens_q[b]), int(lens_k[b])
+    Pq, Pk = (Lq + 127) // 128 * 128, (Lk + 127) // 128 * 128
+    Np = max(Pq, Pk)
+    hk = h // (Hq // Hkv)
+    rq, rk = Hq * int(pq[b]) + h * Pq, Hkv * int(pk[b]) + hk * Pk
+    row_b, tile_b = D // 2, (D // 64) * 512
+    dev = qz["q_fp4"].device
+    dense = {n: torch.zeros(Np * row_b if n.endswith("fp4") else (Np // 128) * tile_b, dtype=torch.uint8,
+                            device=dev) for n in ("q_fp4", "k_fp4", "q_sf", "k_sf")}
+    dense["q_fp4"][: Pq * row_b] = qz["q_fp4"][rq * row_b:(rq + Pq) * row_b]
+    dense["k_fp4"][: Pk * row_b] = qz["k_fp4"][rk * row_b:(rk + Pk) * row_b]
+    dense["q_sf"][: (Pq // 128) * tile_b] = qz["q_sf"][(rq // 128) * tile_b:((rq + Pq) // 128) * tile_b]
+    dense["k_sf"][: (Pk // 128) * tile_b] = qz["k_sf"][(rk // 128) * tile_b:((rk + Pk) // 128) * tile_b]
+    dense.update({"B": 1, "H": 1, "N": Np, "D": D, "Np": Np})
+    s = sage.qk_scores(dense, sm_scale=1.0)
+    torch.cuda.synchronize()
+    return s[0, :Lq, :Lk].double().cpu().numpy()

@@ -55,11 +55,44 @@ def test_traffic_absent_record(bench_mod, tmp_path, monkeypatch):
     assert bench_mod._attn_traffic(W.LONG) == (None, "no capture")
 
 
-def test_committed_record_names_existing_sources(bench_mod):
-    """The committed record names files of the tree; bench reports its figure while they
-    match and null (not an error) once the kernel changed."""
+def test_write_traffic_record_from_ncu_csv(bench_mod, tmp_path, monkeypatch):
+    """The record is written from an ncu CSV (one row per launch and metric, bytes in any
+    of ncu's units) and hashed over the sources as they are when it is written, so that
+    _attn_traffic reports it until a source changes."""
     from microscaling_fp4_quantized_b200 import workloads as W
-    with open(os.path.join(ROOT, "profiles", "attn_fp4_fwd_kernel_traffic.json")) as f:
+    kernel, name, srcs = bench_mod.TRAFFIC_SOURCES[False]
+    for s in srcs:
+        os.makedirs(os.path.dirname(str(tmp_path / s)), exist_ok=True)
+        (tmp_path / s).write_text(f"// {s}\n")
+    os.makedirs(str(tmp_path / "profiles"))
+    head = ('"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream","Section Name",'
+            '"Metric Name","Metric Unit","Metric Value"')
+    rows = [
+        '"0","1","python","h","stats_kernel<128>","1","7","","dram__bytes_read.sum","Mbyte","9.00"',
+        f'"4","1","python","h","void sage::{kernel}<128, false, 0>(...)","1","7","","dram__bytes_read.sum","Mbyte","60.50"',
+        f'"4","1","python","h","void sage::{kernel}<128, false, 0>(...)","1","7","","dram__bytes_write.sum","byte","16,777,216"',
+    ]
+    csv_path = tmp_path / "traffic.csv"
+    csv_path.write_text("==PROF== noise line\n" + head + "\n" + "\n".join(rows) + "\n")
+    monkeypatch.setattr(bench_mod, "ROOT", str(tmp_path))
+    rec = bench_mod.write_traffic_record(str(csv_path), W.PROFILE, False)
+    assert rec["dram_bytes_per_launch"] == pytest.approx(60.5e6 + 16777216)
+    assert rec["launches_captured"] == 1
+    t, src = bench_mod._attn_traffic(W.PROFILE)
+    assert t == pytest.approx(60.5e6 + 16777216) and W.PROFILE.name in src
+    (tmp_path / srcs[0]).write_text("// edited\n")
+    assert bench_mod._attn_traffic(W.PROFILE)[0] is None
+
+
+def test_committed_record_names_existing_sources(bench_mod):
+    """The committed record (if any) names files of the tree; bench reports its figure while
+    they match and null (not an error) once the kernel changed."""
+    from microscaling_fp4_quantized_b200 import workloads as W
+    path = os.path.join(ROOT, "profiles", "attn_fp4_fwd_kernel_traffic.json")
+    if not os.path.exists(path):
+        assert bench_mod._attn_traffic(W.LONG) == (None, "no capture")
+        return
+    with open(path) as f:
         rec = json.load(f)
     for s in rec["sources"]:
         assert os.path.isfile(os.path.join(ROOT, s)), s

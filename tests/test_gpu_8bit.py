@@ -8,7 +8,7 @@ import torch
 
 from gpu_helpers import canonical8, f32
 from microscaling_fp4_quantized_b200 import workloads as W
-from test_gpu_general import _check_rows_over_bar, _out_per_seq, _per_seq
+from test_gpu_general import _out_per_seq, _per_seq
 
 pytestmark = pytest.mark.gpu
 
@@ -103,7 +103,9 @@ def _check_attention8(sage, oracle_mod, w, rows_per_seq=None):
         e = em.reshape(-1, w.D)
         m = oracle_mod.metrics(g, e)
         assert m["cos"] >= MIN_COS, (b, m)
-        _check_rows_over_bar(oracle_mod, w, qs, ks, vs, g, e, rows, MAX_ABS_FRAC * float(np.abs(vs).max()), b)
+        # Every row within the max-abs bar: the 8-bit scores are exact integers, so no
+        # score rounding can move a P~ code here.
+        assert m["max_abs"] <= MAX_ABS_FRAC * float(np.abs(vs).max()), (b, m)
         worst = m if worst is None or m["cos"] < worst["cos"] else worst
     print(f"\n{w.name}: worst sequence vs 8-bit emulation {worst}")
 

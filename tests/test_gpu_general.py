@@ -6,14 +6,15 @@ Quantization: K and Q means within 1 ulp, second-level maxima exact, codes and s
 bytes bit for bit against the oracle fed the GPU's means, Q-smoothing bias within 1e-5
 relative. Attention: the bar of the dense tests (max |O_gpu - O_oracle| <= 1e-2 * max|V|
 and cosine >= 0.999 against the oracle's emulation with the same key-tile width, 128),
-per sequence; a row over the max-abs bar is accepted only as a rare, valid alternative
-result (see _check_rows_over_bar).
+per sequence; a row over the max-abs bar is accepted only when it is rare and the method
+applied by the oracle to the GPU's own FP32 scores of that row reproduces it within the
+bar (see _check_rows_over_bar).
 """
 import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import canonical_problem, f32
+from gpu_helpers import canonical_problem, f32, gpu_row_scores
 from microscaling_fp4_quantized_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -171,24 +172,39 @@ ATTN_CASES = QUANT_CASES + [
 ]
 
 
-def _check_rows_over_bar(oracle_mod, w, qs, ks, vs, g, e, rows, tol, b):
+def _check_rows_over_bar(sage, oracle_mod, w, b, qz_gpu, can_b, qz_or, g, e, rows, tol):
     """Rows whose max-abs difference from the emulation exceeds the bar. P^ codes are not
-    unique (the GPU's FP32 scores round differently from the oracle's binary64 ones), and
+    unique: the GPU's FP32 scores round differently from the oracle's binary64 ones, and
     when attention is strongly peaked one code that flips at a rounding boundary on a
     dominant key moves that row by a few percent of |V|. Such a row is accepted only if it
-    is rare (at most 0.1 % of the rows, one at least) and it is as close to exact
-    attention as the emulated row is, within the same bar."""
-    Lq = qs.shape[1]
+    is rare (at most 0.1 % of the rows, one at least) AND the method, applied by the oracle
+    to that GPU's own FP32 scores of the row (read back through the scores kernel, plus
+    the GPU's own Q-smoothing bias terms), reproduces the GPU row within the bar: the
+    difference then comes from the scores' rounding alone, not from the kernel's softmax,
+    P~ quantization or P^V."""
+    Lq, Lk = w.lens_q[b], w.lens_k[b]
     if rows is None:
         rows = np.array([(h, i) for h in range(w.Hq) for i in range(Lq)], np.int64)
     err = np.abs(g - e).max(axis=1)
     over = np.flatnonzero(err > tol)
     assert len(over) <= max(1, len(err) // 1000), (b, len(over), float(err.max()), tol)
-    if len(over):
-        ex = oracle_mod.attn_exact(qs, ks, vs, w.causal, w.sm_scale, rows=rows[over], heads=(1, w.Hq, w.Hkv))
-        d_gpu = np.abs(g[over] - ex).max(axis=1)
-        d_emu = np.abs(e[over] - ex).max(axis=1)
-        assert (d_gpu <= d_emu + tol).all(), (b, rows[over].tolist(), d_gpu.tolist(), d_emu.tolist(), tol)
+    if not len(over):
+        return
+    group = w.Hq // w.Hkv
+    for o in over:
+        h, i = (int(x) for x in rows[o])
+        acc = gpu_row_scores(sage, qz_gpu, w.lens_q, w.lens_k, w.Hq, w.Hkv, w.D, b, h)[i]
+        if w.smooth_q:
+            acc = acc + can_b["qk_bias"][h]
+        gq = 1.0 if qz_or["gq"] is None else float(qz_or["gq"][h])
+        gk = 1.0 if qz_or["gk"] is None else float(qz_or["gk"][h // group])
+        S = acc * (w.sm_scale * gq * gk)
+        n_keys = min(i + Lk - Lq, Lk - 1) + 1 if w.causal else Lk
+        want = oracle_mod.attn_from_scores(S[None, :], [h // group], [max(n_keys, 0)], qz_or, Bk=BK)[0]
+        d = float(np.abs(g[o] - want).max())
+        print(f"\nsequence {b} row (head {h}, query {i}): {err[o]:.4g} from the emulation, "
+              f"{d:.4g} from the method on the GPU's own scores (bar {tol:.4g})")
+        assert d <= tol, (b, h, i, d, float(err[o]), tol)
 
 
 def _check_attention(sage, oracle_mod, w, rows_per_seq=None):
@@ -220,17 +236,17 @@ def _check_attention(sage, oracle_mod, w, rows_per_seq=None):
             heads = sorted({0, w.Hq - 1})
             rr = np.unique(np.concatenate([[0, Lq - 1], rng.choice(Lq, min(Lq, rows_per_seq), replace=False)]))
             rows = np.array([(h, i) for h in heads for i in rr], np.int64)
-        em, _ = oracle_mod.attention(qs, ks, vs, w.causal, w.sm_scale, Bk=BK, rows=rows,
-                                     kmean_in=kmeans[b], gscale=w.gscale, heads=(1, w.Hq, w.Hkv),
-                                     amax_in=amax_t[b], smooth_q=w.smooth_q,
-                                     qmean_in=qmeans[b] if w.smooth_q else None)
+        em, qz_or = oracle_mod.attention(qs, ks, vs, w.causal, w.sm_scale, Bk=BK, rows=rows,
+                                         kmean_in=kmeans[b], gscale=w.gscale, heads=(1, w.Hq, w.Hkv),
+                                         amax_in=amax_t[b], smooth_q=w.smooth_q,
+                                         qmean_in=qmeans[b] if w.smooth_q else None)
         g = got.reshape(-1, w.D) if rows is None else got[rows[:, 0], rows[:, 1]]
         e = em.reshape(-1, w.D)
         m = oracle_mod.metrics(g, e)
         vmax = float(np.abs(vs).max())
         tol = MAX_ABS_FRAC * vmax
         assert m["cos"] >= MIN_COS, (b, m)
-        _check_rows_over_bar(oracle_mod, w, qs, ks, vs, g, e, rows, tol, b)
+        _check_rows_over_bar(sage, oracle_mod, w, b, qz, can[b], qz_or, g, e, rows, tol)
         worst = m if worst is None or m["cos"] < worst["cos"] else worst
     print(f"\n{w.name}: worst sequence vs emulated {worst}")
 

@@ -200,3 +200,34 @@ def test_emulated_close_to_exact_on_tiny_workload(oracle_mod):
     # cancelling average, so FP4 error is large relative to |O|: Q,K,V quantization
     # alone measures cos ~0.985 here. 0.97 only guards against gross breakage.
     assert m["cos"] > 0.97, m
+
+
+@pytest.mark.parametrize("causal,Nq,Nk,gscale", [(False, 130, 300, "none"), (True, 300, 300, "head"),
+                                                  (True, 100, 260, "none"), (True, 260, 100, "tensor")])
+def test_attn_from_scores_equals_emulation(oracle_mod, causal, Nq, Nk, gscale):
+    # The emulation's tile walk applied to given scores: fed the emulation's own scores
+    # (formed here in numpy from the dequantized codes; products of E2M1 codes and E4M3
+    # scales are exact in binary64, and so are their sums at these sizes), it must give
+    # the emulated rows bit for bit, for grouped heads and masks. With a second-level
+    # scale the products carry a 24-bit factor and are rounded in another order, so the
+    # rows agree to binary64 rounding instead.
+    Hq, Hkv, D, sm = 4, 2, 64, 0.125
+    rng = np.random.default_rng(Nq + Nk)
+    q = rng.standard_normal((Hq, Nq, D)).astype(np.float32)
+    k = (rng.standard_normal((Hkv, Nk, D)) + 1.5).astype(np.float32)
+    v = rng.standard_normal((Hkv, Nk, D)).astype(np.float32)
+    em, qz = oracle_mod.attention(q, k, v, causal, sm, gscale=gscale, heads=(1, Hq, Hkv))
+    dec = lambda c, s: oracle_mod.e2m1_decode(oracle_mod.unpack_fp4(c)) * np.repeat(oracle_mod.e4m3_decode(s), 16, -1)  # noqa: E731
+    qd, kd = dec(qz["q_codes"], qz["q_sf"]), dec(qz["k_codes"], qz["k_sf"])
+    gq = np.ones(Hq) if qz["gq"] is None else qz["gq"].astype(np.float64)
+    gk = np.ones(Hkv) if qz["gk"] is None else qz["gk"].astype(np.float64)
+    for h in range(Hq):
+        hk = h // (Hq // Hkv)
+        S = sm * np.einsum("id,jd->ij", qd[h] * gq[h], kd[hk] * gk[hk])
+        n_keys = [min(i + Nk - Nq, Nk - 1) + 1 if causal else Nk for i in range(Nq)]
+        n_keys = [max(n, 0) for n in n_keys]
+        got = oracle_mod.attn_from_scores(S, [hk] * Nq, n_keys, qz)
+        if gscale == "none":
+            assert np.array_equal(got, em[h]), h
+        else:
+            assert np.abs(got - em[h]).max() <= 1e-12 * np.abs(v).max(), h

@@ -216,3 +216,78 @@ def test_varlen_tensor_scale_spans_all_sequences(oracle_mod):
                                           smooth_k=False, rows=rows)
     assert np.array_equal(part, out[rows[:, 0], rows[:, 1]])
     assert math.isfinite(float(np.abs(out).max()))
+
+
+def _separate_sequences(lq, lk, Hq, Hkv, D, seed):
+    """Each sequence drawn on its own as [H, L, D] arrays (never sliced from a packed
+    tensor), then packed by concatenation along tokens into [T, H, D]."""
+    rng = np.random.default_rng(seed)
+    seqs = []
+    for b, (a, c) in enumerate(zip(lq, lk)):
+        q = rng.standard_normal((Hq, a, D)).astype(np.float32)
+        k = (rng.standard_normal((Hkv, c, D)) + rng.normal(0, 2, (Hkv, 1, D))).astype(np.float32)
+        v = rng.standard_normal((Hkv, c, D)).astype(np.float32)
+        seqs.append((q, k, v))
+    pack = lambda i, H: np.concatenate([s[i].transpose(1, 0, 2) for s in seqs], 0).reshape(-1, H, D)  # noqa: E731
+    cu_q = np.concatenate([[0], np.cumsum(lq)]).astype(np.int64)
+    cu_k = np.concatenate([[0], np.cumsum(lk)]).astype(np.int64)
+    return seqs, pack(0, Hq), pack(1, Hkv), pack(2, Hkv), cu_q, cu_k
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("gscale,smooth_q", [("none", False), ("head", False), ("none", True)])
+def test_varlen_equals_each_sequence_alone(oracle_mod, causal, gscale, smooth_q):
+    # Every sequence is its own problem with its own K mean (and query mean, and
+    # per-(sequence, head) scales): the packed result must equal oracle.attention on each
+    # separately drawn sequence, bit for bit, and zero rows for a sequence with no keys.
+    Hq, Hkv, D = 4, 2, 64
+    lq, lk = [130, 1, 0, 77, 40], [200, 5, 3, 77, 0]
+    seqs, q, k, v, cu_q, cu_k = _separate_sequences(lq, lk, Hq, Hkv, D, 31)
+    got, _ = oracle_mod.attention_varlen(q, k, v, cu_q, cu_k, causal, 0.125, gscale=gscale,
+                                         smooth_q=smooth_q)
+    for b, (qs, ks, vs) in enumerate(seqs):
+        seg = got[cu_q[b]:cu_q[b + 1]]
+        if lq[b] == 0:
+            assert seg.shape[0] == 0
+            continue
+        if lk[b] == 0:
+            assert not seg.any()
+            continue
+        want, _ = oracle_mod.attention(qs, ks, vs, causal, 0.125, gscale=gscale, heads=(1, Hq, Hkv),
+                                       smooth_q=smooth_q)
+        assert np.array_equal(seg.transpose(1, 0, 2), want), b
+    # Sampled (token, head) rows equal the same rows of the full result.
+    rows = np.array([[0, 0], [129, 3], [130, 1], [131 + 76, 2], [131 + 77 + 39, 0]])
+    part, _ = oracle_mod.attention_varlen(q, k, v, cu_q, cu_k, causal, 0.125, gscale=gscale,
+                                          smooth_q=smooth_q, rows=rows)
+    assert np.array_equal(part, got[rows[:, 0], rows[:, 1]])
+
+
+def test_varlen_equal_lengths_equal_dense_batches(oracle_mod):
+    # With every length equal, the packed problem is the dense [B, H, N, D] problem: the
+    # dense oracle indexes batches itself (per-(batch, head) K means inside the C code),
+    # the packed one slices sequences in Python, and they must agree bit for bit.
+    B, Hq, Hkv, N, D = 3, 4, 2, 150, 64
+    seqs, q, k, v, cu_q, cu_k = _separate_sequences([N] * B, [N] * B, Hq, Hkv, D, 32)
+    got, _ = oracle_mod.attention_varlen(q, k, v, cu_q, cu_k, True, 0.125)
+    qd = np.concatenate([s[0] for s in seqs], 0)
+    kd = np.concatenate([s[1] for s in seqs], 0)
+    vd = np.concatenate([s[2] for s in seqs], 0)
+    dense, _ = oracle_mod.attention(qd, kd, vd, True, 0.125, heads=(B, Hq, Hkv))
+    assert np.array_equal(got.reshape(B, N, Hq, D).transpose(0, 2, 1, 3).reshape(B * Hq, N, D), dense)
+
+
+def test_varlen_tensor_scale_is_the_plain_maximum(oracle_mod):
+    # The per-tensor second-level maxima are max |x| over every sequence and head (K after
+    # subtracting its own sequence's mean), computed here directly with numpy.
+    Hq, Hkv, D = 2, 1, 64
+    lq, lk = [60, 33], [50, 90]
+    seqs, q, k, v, cu_q, cu_k = _separate_sequences(lq, lk, Hq, Hkv, D, 33)
+    a = oracle_mod.varlen_amax(q, k, v, cu_q, cu_k)
+    want_q = max(np.abs(s[0]).max() for s in seqs)
+    want_v = max(np.abs(s[2]).max() for s in seqs)
+    want_k = 0.0
+    for _, ks, _ in seqs:
+        mu = (ks.astype(np.float64).sum(1) / ks.shape[1]).astype(np.float32)
+        want_k = max(want_k, float(np.abs((ks - mu[:, None, :]).astype(np.float32)).max()))
+    assert a["q"] == np.float32(want_q) and a["v"] == np.float32(want_v) and a["k"] == np.float32(want_k)
