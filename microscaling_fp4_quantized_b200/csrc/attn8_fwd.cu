@@ -126,13 +126,6 @@ __device__ __forceinline__ float s32_to_f32(uint32_t raw) {
   return __uint_as_float(raw + 0x4B400000u) - 12582912.0f;
 }
 
-// E4M3 bytes of two non-negative floats (RNE, saturating); lo lands in the low byte.
-__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
 }  // namespace
 
 template <int D, bool CAUSAL>

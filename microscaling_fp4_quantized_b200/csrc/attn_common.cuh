@@ -63,6 +63,17 @@ __device__ __forceinline__ void tmem_wait_regs(uint32_t (&r)[32]) {
       : "memory");
 }
 
+// 16 columns from TMEM, with the wait::ld tied to the registers it produces.
+__device__ __forceinline__ void tmem_wait_regs16(uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+        "+r"(r[14]), "+r"(r[15])
+      :
+      : "memory");
+}
+
 __device__ __forceinline__ void store_out8(void* out, size_t idx, const float* v, int dtype) {
   uint4 w;
   uint32_t* ww = reinterpret_cast<uint32_t*>(&w);

@@ -10,10 +10,11 @@ namespace sage {
 namespace {
 
 template <int D>
-cudaError_t launch_attn_full_d(const TensorMaps& m, const AttnParams& p, int tiles_q, int mode, cudaStream_t stream) {
-  if (mode == 2) return launch_attn_t<D, false, 2>(m, p, tiles_q, stream);
-  if (mode == 1) return launch_attn_t<D, false, 1>(m, p, tiles_q, stream);
-  return launch_attn_t<D, false, 0>(m, p, tiles_q, stream);
+cudaError_t launch_attn_full_d(const TensorMaps& m, const AttnParams& p, int tiles_q, int mode, int max_ctas,
+                               cudaStream_t stream) {
+  if (mode == 2) return launch_attn_t<D, false, 2>(m, p, tiles_q, max_ctas, stream);
+  if (mode == 1) return launch_attn_t<D, false, 1>(m, p, tiles_q, max_ctas, stream);
+  return launch_attn_t<D, false, 0>(m, p, tiles_q, max_ctas, stream);
 }
 
 }  // namespace
@@ -25,12 +26,18 @@ cudaError_t launch_attention(const TensorMaps& m, const AttnParams& p, int tiles
   // gets the leaner loop (constant score scale, no mask offset, no empty-row guard).
   const bool general = p.seq.cu_q != nullptr || p.seq.Nq != p.seq.Nk || p.amax != nullptr;
   const int mode = p.qk_bias != nullptr ? 2 : (general ? 1 : 0);
-  if (p.causal) return launch_attention_causal(m, p, tiles_q, mode, stream);
-  // Few query tiles per (sequence, head): the persistent form hides each CTA's start-up
-  // (measured at D = 128: 805 against 727 TFLOP/s on B64 H32 N1024; long rows unchanged).
-  if (mode == 0 && p.D == 128 && tiles_q <= kShortTiles) return launch_attention_short(m, p, tiles_q, stream);
-  return p.D == 64 ? launch_attn_full_d<64>(m, p, tiles_q, mode, stream)
-                   : launch_attn_full_d<128>(m, p, tiles_q, mode, stream);
+  // Few query tiles per (sequence, head): one CTA per SM walks the work items, which
+  // hides each CTA's start-up and drain; otherwise one CTA per item.
+  int max_ctas = 0;
+  if (tiles_q <= kShortTiles) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&max_ctas, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+  }
+  if (p.causal) return launch_attention_causal(m, p, tiles_q, mode, max_ctas, stream);
+  return p.D == 64 ? launch_attn_full_d<64>(m, p, tiles_q, mode, max_ctas, stream)
+                   : launch_attn_full_d<128>(m, p, tiles_q, mode, max_ctas, stream);
 }
 
 // S = sm_scale * Q^ K^^T for one (query tile, key tile, head): the QK^T stage alone.

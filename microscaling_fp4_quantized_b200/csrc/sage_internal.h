@@ -158,7 +158,7 @@ struct AttnParams {
   uint32_t* err;        // device error word
   uint64_t timeout_ns;  // bound on every wait
   uint32_t debug_flags; // kDebugNoLoads: the producer issues no copies (test of the error path)
-  int tiles_q;          // query tiles of the longest sequence (set by the persistent launcher)
+  int tiles_q;          // query tiles of the longest sequence (work items: B * Hq * tiles_q)
 };
 
 enum : uint32_t { kDebugNoLoads = 1u };
@@ -176,9 +176,8 @@ cudaError_t launch_quantize8(const QuantParams& p, const QuantLaunch& l, cudaStr
 cudaError_t launch_attention(const TensorMaps& maps, const AttnParams& p, int tiles_q, cudaStream_t stream);
 cudaError_t launch_qk_scores(const TensorMaps& maps, const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_attention8(const TensorMaps& maps, const AttnParams& p, int tiles_q, cudaStream_t stream);
-// The persistent FP4 attention kernel (square dense, one-level scales, non-causal), used
-// by launch_attention at D = 128 when there are at most kShortTiles query tiles.
-cudaError_t launch_attention_short(const TensorMaps& maps, const AttnParams& p, int tiles_q, cudaStream_t stream);
+// Up to this many query tiles per (sequence, head), launch_attention runs one CTA per SM
+// over all work items instead of one CTA per item.
 constexpr int kShortTiles = 8;
 // Tensor-core rate probe (mma_rate.cu): `ctas` CTAs, each issuing `iters` block-scaled FP4
 // products of M = 128, N = n, K = 64.

@@ -295,6 +295,13 @@ __device__ __forceinline__ uint32_t f32_to_e4m3(float x) {
   return r & 0xFFu;
 }
 
+// E4M3 (RNE, saturating) bytes of two non-negative floats: `lo` in bits 0-7, `hi` in 8-15.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 __device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
   uint32_t h2;
   const uint16_t in = static_cast<uint16_t>(b & 0xFFu);
