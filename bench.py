@@ -7,12 +7,16 @@ ranks. The inputs (576 MiB) exceed the 126 MB L2, so no flush runs between steps
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-Under torchrun each rank runs its own copy of the workload (independent problems: weak
-scaling, no data-path collective); the time is the max over ranks.
+Under torchrun the job is one problem of world x B*H (batch, head) pairs split across the
+ranks by microscaling_fp4_quantized_b200.shard.head_slice: rank r holds and computes its
+own contiguous slice (the workload's shape, drawn with the rank's own seed). The pairs are
+independent, so there is no data-path collective (weak scaling: the work per GPU is
+fixed); the time is the max over ranks.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -205,7 +209,7 @@ def max_over_ranks(value: float, dist, device) -> float:
 
 
 def job_value(ops_per_rank: float, world: int, ms_per_step: float) -> float:
-    """Whole-job throughput in TOPS: every rank runs its own copy of the workload."""
+    """Whole-job throughput in TOPS: every rank computes its slice of ops_per_rank."""
     return world * ops_per_rank / (ms_per_step * 1e-3) / 1e12
 
 
@@ -515,7 +519,8 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    q, k, v = workloads.make_inputs(wl)          # CPU, seeded
+    # This rank's slice of the global problem: the workload's shape, its own seed.
+    q, k, v = workloads.make_inputs(dataclasses.replace(wl, seed=wl.seed + 1000 * rank) if rank else wl)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     out = torch.empty_like(qd)
     plan = sage.ProblemPlan(sage.sageattn_problem(qd, kd, vd, out, "HND", wl.causal, wl.sm_scale,
