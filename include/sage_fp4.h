@@ -87,7 +87,9 @@ typedef enum {
                                (from sage_fp4_get_device_error) a bad sequence table */
   SAGE_ERR_UNSUPPORTED = 2, /* D not in {64, 128}, or a size beyond the 32-bit indexing limits */
   SAGE_ERR_CUDA = 3,        /* a CUDA runtime/driver call or launch failed */
-  SAGE_ERR_TIMEOUT = 4      /* a bounded wait inside a kernel ran out (see above) */
+  SAGE_ERR_TIMEOUT = 4,     /* a bounded wait inside a kernel ran out (see above) */
+  SAGE_ERR_BOUNDS = 5       /* bounds-checked build only: a kernel refused an out-of-range
+                               index (an internal error; the access was skipped) */
 } sage_status_t;
 
 typedef enum { SAGE_BF16 = 0, SAGE_F16 = 1 } sage_dtype_t;
@@ -301,9 +303,11 @@ const char* sage_fp4_last_cuda_error(void);
  * Test switch for the error path (0 = normal operation, the default). Bit 0: the
  * attention kernel's copy warp issues no loads, so every wait of the other roles runs
  * out after the bound set below; the kernel then drains, frees its tensor memory and
- * returns, and sage_fp4_get_device_error() reports SAGE_ERR_TIMEOUT. Nothing faults and
- * nothing waits without bound. Applies to launches made after the call; other bits are
- * rejected with SAGE_ERR_INVALID_ARG.
+ * returns, and sage_fp4_get_device_error() reports SAGE_ERR_TIMEOUT. Bit 1 (bounds-checked
+ * build only, else SAGE_ERR_UNSUPPORTED): the attention kernels take the output's extent
+ * as 0, so every output store fails its check, is skipped and reported (SAGE_ERR_BOUNDS).
+ * Nothing faults and nothing waits without bound. Applies to launches made after the
+ * call; other bits are rejected with SAGE_ERR_INVALID_ARG.
  */
 sage_status_t sage_fp4_set_debug_flags(uint32_t flags);
 
@@ -319,6 +323,18 @@ sage_status_t sage_fp4_set_debug_flags(uint32_t flags);
  * memory; the products themselves are discarded.
  */
 sage_status_t sage_fp4_mma_rate(int n, int iters, int ctas, void* stream);
+
+/*
+ * 1 when this library is the bounds-checked build (libsage_fp4_checks.so, compiled with
+ * SAGE_CHECKS): every computed global index of the quantization and attention kernels --
+ * input rows, quantized codes and scale tiles, statistics, TMA rows, the output -- is
+ * tested against the extents the problem implies before the access; a failure sets a bit
+ * of the device error word (sage_fp4_get_device_error returns SAGE_ERR_BOUNDS), raises the
+ * CTA's abort flag where the kernel has one, and skips the access (no trap). 0 for the
+ * regular build, where the checks compile to nothing. A debugging stand-in for a memory
+ * checker; slower than the regular build.
+ */
+int sage_fp4_bounds_checked(void);
 
 /*
  * Bound on every in-kernel wait, in nanoseconds (default 2e9; 0 restores the default).

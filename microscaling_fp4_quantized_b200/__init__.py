@@ -26,7 +26,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 # SAGE_FP4_LIB may point at another build of the same library (A/B comparisons).
 LIB_PATH = os.environ.get("SAGE_FP4_LIB") or os.path.join(_HERE, "libsage_fp4.so")
 
-SAGE_OK, SAGE_ERR_INVALID_ARG, SAGE_ERR_UNSUPPORTED, SAGE_ERR_CUDA, SAGE_ERR_TIMEOUT = range(5)
+SAGE_OK, SAGE_ERR_INVALID_ARG, SAGE_ERR_UNSUPPORTED, SAGE_ERR_CUDA, SAGE_ERR_TIMEOUT, SAGE_ERR_BOUNDS = range(6)
 SAGE_BF16, SAGE_F16 = 0, 1
 GSCALE = {"none": 0, "tensor": 1, "head": 2}
 PRECISION = {"fp4": 0, "8bit": 1}
@@ -38,6 +38,7 @@ EXPORTED = [
     "sage_fp4_get_device_error", "sage_fp4_set_wait_timeout_ns", "sage_fp4_attn_fwd_noalloc",
     "sage_fp4_last_cuda_error", "sage_fp4_set_debug_flags", "sage_fp4_problem_sizes",
     "sage_fp4_quantize", "sage_fp4_attn_quantized", "sage_fp4_attn", "sage_fp4_mma_rate",
+    "sage_fp4_bounds_checked",
 ]
 
 
@@ -120,6 +121,7 @@ def lib():
         L.sage_fp4_attn_quantized.argtypes = [pp, ctypes.POINTER(_Quantized), vp, vp]
         L.sage_fp4_attn.argtypes = [pp, vp, vp, vp, vp, vp, sz, vp]
         L.sage_fp4_mma_rate.argtypes = [i, i, i, vp]
+        L.sage_fp4_bounds_checked.argtypes = []
         for n in EXPORTED[1:]:
             if n not in ("sage_fp4_quantize_scratch_bytes", "sage_fp4_workspace_bytes",
                          "sage_fp4_last_cuda_error"):
@@ -270,7 +272,7 @@ def qk_scores(qz: dict, sm_scale: Optional[float] = None) -> torch.Tensor:
     return s
 
 
-DEV_ERR_TIMEOUT, DEV_ERR_SEQLENS = 1, 2
+DEV_ERR_TIMEOUT, DEV_ERR_SEQLENS, DEV_ERR_BOUNDS = 1, 2, 4
 
 
 def device_error(device=None) -> int:
@@ -278,7 +280,7 @@ def device_error(device=None) -> int:
     bounded wait ran out, bit 1 a packed problem's sequence table failed its check."""
     w = ctypes.c_uint32(0)
     st = lib().sage_fp4_get_device_error(ctypes.byref(w), _stream(device))
-    if st not in (SAGE_OK, SAGE_ERR_TIMEOUT, SAGE_ERR_INVALID_ARG):
+    if st not in (SAGE_OK, SAGE_ERR_TIMEOUT, SAGE_ERR_INVALID_ARG, SAGE_ERR_BOUNDS):
         raise SageError(st, "sage_fp4_get_device_error")
     return int(w.value)
 

@@ -199,12 +199,18 @@ __global__ void __launch_bounds__(kThreads8, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer ----
     if (lane == 0 && !(p.debug_flags & kDebugNoLoads)) {
-      mbar_arrive_expect_tx(bar(E_QFULL), L::kQBytes);
-      tma_load_2d(sbase + L::off_q, &tm_q, 0, qrow0, bar(E_QFULL));
+      const bool q_in = SAGE_IN_BOUNDS(static_cast<uint64_t>(qrow0) + 128 <= p.lim.rows_q, p.err, ctl.abort);
+      if (q_in) {
+        mbar_arrive_expect_tx(bar(E_QFULL), L::kQBytes);
+        tma_load_2d(sbase + L::off_q, &tm_q, 0, qrow0, bar(E_QFULL));
+      }
       int issued = 0;
-      for (int j = 0; j < nt; ++j) {
+      for (int j = 0; q_in && j < nt; ++j) {
         const int st = j % kStages8;
         if (!wait_bar(bar(E_KVEMPTY + st), ((j / kStages8) & 1) ^ 1, ctl)) break;
+        if (!SAGE_IN_BOUNDS(static_cast<uint64_t>(ktile0 + j + 1) * 128 <= p.lim.rows_k &&
+                                static_cast<uint64_t>(ktile0 + j + 1) * D <= p.lim.rows_v,
+                            p.err, ctl.abort)) break;
         const uint32_t sst = sbase + L::off_stage + st * L::kStageBytes;
         mbar_arrive_expect_tx(bar(E_KFULL + st), L::kKBytes);
         tma_load_2d(sst + L::st_k, &tm_k, 0, (ktile0 + j) * 128, bar(E_KFULL + st));
@@ -216,7 +222,7 @@ __global__ void __launch_bounds__(kThreads8, 1)
         // Let every copy this thread started land before the CTA releases its memory.
         Ctl drain{misc + 2, p.err, p.timeout_ns};
         misc[2] = 0u;
-        wait_bar(bar(E_QFULL), 0, drain);
+        if (q_in) wait_bar(bar(E_QFULL), 0, drain);
         for (int j = (issued > kStages8 ? issued - kStages8 : 0); j < issued; ++j) {
           wait_bar(bar(E_KFULL + j % kStages8), (j / kStages8) & 1, drain);
           wait_bar(bar(E_VFULL + j % kStages8), (j / kStages8) & 1, drain);
@@ -415,7 +421,7 @@ __global__ void __launch_bounds__(kThreads8, 1)
         float v8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) v8[i] = o[d + i] * il * sc[i];
-        store_out8(p.out, base + d, v8, p.out_dtype);
+        if (SAGE_IN_BOUNDS(base + d + 8 <= p.lim.o_el, p.err, nullptr)) store_out8(p.out, base + d, v8, p.out_dtype);
       }
     }
   }

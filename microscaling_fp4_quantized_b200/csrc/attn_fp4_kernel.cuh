@@ -334,6 +334,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!it.valid || it.nt == 0) continue;
         const int qs = qi % kQSlots;
         if (!wait_bar(bar(B_QEMPTY + qs), ((qi / kQSlots) & 1) ^ 1, ctl, kIdleNs, kCheck)) { ok = false; break; }
+        if (!SAGE_IN_BOUNDS(static_cast<uint64_t>(it.qrow0) + 128 <= p.lim.rows_q &&
+                                static_cast<uint64_t>((it.qrow0 >> 7) + 1) * L::kSfQKBytes <= p.lim.q_sf,
+                            p.err, ctl.abort)) { ok = false; break; }
         const uint32_t sq = sbase + L::off_q + qs * L::kQSlotBytes;
         mbar_arrive_expect_tx(bar(B_QFULL + qs), L::kQBytes + L::kSfQKBytes);
         tma_load_2d(sq, &tm_q, 0, it.qrow0, bar(B_QFULL + qs));
@@ -344,6 +347,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int st = gt % kKStages;
           if (!wait_bar(bar(B_KEMPTY + st), ((gt / kKStages) & 1) ^ 1, ctl, kIdleNs, kCheck)) { ok = false; break; }
           const uint32_t sst = sbase + L::off_stage + st * L::kKStageBytes;
+          if (!SAGE_IN_BOUNDS(static_cast<uint64_t>(it.ktile0 + j + 1) * 128 <= p.lim.rows_k &&
+                                  static_cast<uint64_t>(it.ktile0 + j + 1) * L::kSfQKBytes <= p.lim.k_sf &&
+                                  (!QBIAS || (it.bias_row0 + static_cast<size_t>(j + 1) * 128) * 32 <= p.lim.qk_bias),
+                              p.err, ctl.abort)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(B_KFULL + st), L::kKBytes + L::kSfQKBytes + L::kBiasBytes);
           tma_load_2d(sst + L::st_k, &tm_k, 0, (it.ktile0 + j) * 128, bar(B_KFULL + st));
           bulk_load(sst + L::st_sfk, p.k_sf + static_cast<size_t>(it.ktile0 + j) * L::kSfQKBytes,
@@ -377,6 +384,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int st = gt % kVStages;
           if (!wait_bar(bar(B_VEMPTY + st), ((gt / kVStages) & 1) ^ 1, ctl, kIdleNs, kCheck)) { ok = false; break; }
           const uint32_t sst = sbase + L::off_vstage + st * L::kVStageBytes;
+          if (!SAGE_IN_BOUNDS(static_cast<uint64_t>(it.ktile0 + j + 1) * D <= p.lim.rows_v &&
+                                  static_cast<uint64_t>(it.ktile0 + j + 1) * L::kSfVBytes <= p.lim.vt_sf,
+                              p.err, ctl.abort)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(B_VFULL + st), L::kVBytes + L::kSfVBytes);
           tma_load_2d(sst + L::st_v, &tm_v, 0, (it.ktile0 + j) * D, bar(B_VFULL + st));
           bulk_load(sst + L::st_sfv, p.vt_sf + static_cast<size_t>(it.ktile0 + j) * L::kSfVBytes,
@@ -563,7 +573,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           float v8[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) v8[i] = o[d + i] * il;
-          store_out8(p.out, base + d, v8, p.out_dtype);
+          if (SAGE_IN_BOUNDS(base + d + 8 <= p.lim.o_el, p.err, nullptr)) store_out8(p.out, base + d, v8, p.out_dtype);
         }
       }
     }  // work items

@@ -122,6 +122,17 @@ __device__ __forceinline__ const char* row_ptr(const void* base, const Strides& 
   return static_cast<const char*>(base) + (static_cast<int64_t>(b) * s.b + static_cast<int64_t>(h) * s.h + tok * s.n) * 2;
 }
 
+// 16 bytes (8 elements, channels 8c .. 8c + 7) of row (b, h, tok) of a caller tensor;
+// the bounds-checked build refuses an offset outside the problem's extent (zeros).
+__device__ __forceinline__ uint4 ld_row16(const void* base, const Strides& s, int b, int h, int64_t tok, int c,
+                                          uint64_t lim_el, uint32_t* err) {
+  const int64_t off = static_cast<int64_t>(b) * s.b + static_cast<int64_t>(h) * s.h + tok * s.n + 8 * c;
+  (void)lim_el;
+  (void)err;
+  if (!SAGE_IN_BOUNDS(off >= 0 && static_cast<uint64_t>(off) + 8 <= lim_el, err, nullptr)) return make_uint4(0, 0, 0, 0);
+  return ld_nc_16(static_cast<const char*>(base) + off * 2);
+}
+
 __device__ __forceinline__ float block_max(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -217,7 +228,8 @@ template <int D>
 __device__ __forceinline__ void chunk_channel_stats(const void* src, const Strides& st, int dtype, int b, int h,
                                                     int64_t tok0, int n0, int n1, bool extremes,
                                                     double* sum, float* cmax, float* cmin,
-                                                    double (*red)[D], float (*redmx)[D], float (*redmn)[D]) {
+                                                    double (*red)[D], float (*redmx)[D], float (*redmn)[D],
+                                                    uint64_t lim_el, uint32_t* err) {
   constexpr int CPR = D / 8;
   constexpr int RG = kThreads / CPR;
   const int t = threadIdx.x, c = t % CPR, rg = t / CPR;
@@ -232,7 +244,7 @@ __device__ __forceinline__ void chunk_channel_stats(const void* src, const Strid
 #pragma unroll 8
   for (int n = n0 + rg; n < n1; n += RG) {
     float x[8];
-    unpack8(ld_nc_16(row_ptr(src, st, b, h, tok0 + n) + c * 16), dtype, x);
+    unpack8(ld_row16(src, st, b, h, tok0 + n, c, lim_el, err), dtype, x);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       acc[e] += static_cast<double>(x[e]);
@@ -287,20 +299,23 @@ __global__ void __launch_bounds__(kThreads, 4) stats_kernel(QuantParams p) {
 
   if (h < p.Hkv && (p.smooth_k || gs) && n0 < si.len_k) {
     const size_t base = (static_cast<size_t>(b * p.Hkv + h) * p.nsplit + split) * D;
+    if (!SAGE_IN_BOUNDS(base + D <= p.lim.stat_el, p.err, nullptr)) return;
     chunk_channel_stats<D>(p.k, p.sk, p.dtype, b, h, si.tok_k, n0, min(n0 + kChunk, si.len_k), gs,
                            p.ksum + base, gs ? p.kmax + base : nullptr, gs ? p.kmin + base : nullptr,
-                           red, redmx, redmn);
+                           red, redmx, redmn, p.lim.k_el, p.err);
   }
   if (h < p.Hkv && p.bits8 && n0 < si.len_k) {
     const size_t base = (static_cast<size_t>(b * p.Hkv + h) * p.nsplit + split) * D;
+    if (!SAGE_IN_BOUNDS(base + D <= p.lim.stat_el, p.err, nullptr)) return;
     chunk_channel_stats<D>(p.v, p.sv, p.dtype, b, h, si.tok_k, n0, min(n0 + kChunk, si.len_k), true,
-                           p.vsum + base, p.vmax + base, p.vmin + base, red, redmx, redmn);
+                           p.vsum + base, p.vmax + base, p.vmin + base, red, redmx, redmn, p.lim.v_el, p.err);
   }
   if (h < p.Hq && p.smooth_q && n0 < si.len_q) {
     const size_t base = (static_cast<size_t>(b * p.Hq + h) * p.nsplit + split) * D;
+    if (!SAGE_IN_BOUNDS(base + D <= p.lim.qstat_el, p.err, nullptr)) return;
     chunk_channel_stats<D>(p.q, p.sq, p.dtype, b, h, si.tok_q, n0, min(n0 + kChunk, si.len_q), gs,
                            p.qsum + base, gs ? p.qmax + base : nullptr, gs ? p.qmin + base : nullptr,
-                           red, redmx, redmn);
+                           red, redmx, redmn, p.lim.q_el, p.err);
   }
   if (!gs) return;
   for (int job = 0; job < 2; ++job) {  // 0: Q (unsmoothed), 1: V
@@ -316,12 +331,14 @@ __global__ void __launch_bounds__(kThreads, 4) stats_kernel(QuantParams p) {
 #pragma unroll 8
     for (int n = n0 + rg; n < n1; n += RG) {
       float x[8];
-      unpack8(ld_nc_16(row_ptr(src, st, b, h, static_cast<int64_t>(tok) + n) + c * 16), p.dtype, x);
+      unpack8(ld_row16(src, st, b, h, static_cast<int64_t>(tok) + n, c, job == 0 ? p.lim.q_el : p.lim.v_el, p.err), p.dtype, x);
 #pragma unroll
       for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(x[e]));
     }
     a = block_max(a, redw);
-    if (t == 0) (job == 0 ? p.qamax : p.vamax)[static_cast<size_t>(b * H + h) * p.nsplit + split] = a;
+    const size_t ia = static_cast<size_t>(b * H + h) * p.nsplit + split;
+    if (t == 0 && SAGE_IN_BOUNDS(ia < (job == 0 ? p.lim.qamax_el : p.lim.vamax_el), p.err, nullptr))
+      (job == 0 ? p.qamax : p.vamax)[ia] = a;
   }
 }
 
@@ -344,7 +361,8 @@ __global__ void __launch_bounds__(D) finalize_kernel(QuantParams p) {
       for (int g = 0; g < ns; ++g) s += p.ksum[base + static_cast<size_t>(g) * D];
       mu = static_cast<float>(s / static_cast<double>(si.len_k));
     }
-    p.k_mean[static_cast<size_t>(b * p.Hkv + h) * D + d] = mu;
+    if (SAGE_IN_BOUNDS(static_cast<size_t>(b * p.Hkv + h) * D + d < p.lim.k_mean_el, p.err, nullptr))
+      p.k_mean[static_cast<size_t>(b * p.Hkv + h) * D + d] = mu;
     if (p.bits8) {
       // E4M3 scale of V's channel d: fp32(max |v| / 448) over the sequence's tokens.
       float mx = -INFINITY, mn = INFINITY;
@@ -386,7 +404,8 @@ __global__ void __launch_bounds__(D) finalize_kernel(QuantParams p) {
         for (int g = 0; g < ns; ++g) s += p.qsum[base + static_cast<size_t>(g) * D];
         mu = static_cast<float>(s / static_cast<double>(si.len_q));
       }
-      p.q_mean[static_cast<size_t>(b * p.Hq + h) * D + d] = mu;
+      if (SAGE_IN_BOUNDS(static_cast<size_t>(b * p.Hq + h) * D + d < p.lim.q_mean_el, p.err, nullptr))
+        p.q_mean[static_cast<size_t>(b * p.Hq + h) * D + d] = mu;
       if (gs && si.len_q > 0) {
         float mx = -INFINITY, mn = INFINITY;
         for (int g = 0; g < ns; ++g) {
@@ -462,7 +481,8 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(QuantParams p) {
 #pragma unroll
     for (int it = 0; it < kIter; ++it) {
       const int rl = rl0 + it * kRowStep;
-      raw[it] = rl < rows ? ld_nc_16(row_ptr(src, st, b, h, tok0 + rl) + c * 16) : make_uint4(0, 0, 0, 0);
+      raw[it] = rl < rows ? ld_row16(src, st, b, h, tok0 + rl, c, job == 0 ? p.lim.q_el : p.lim.k_el, p.err)
+                          : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int it = 0; it < kIter; ++it) {
@@ -509,8 +529,10 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(QuantParams p) {
             uint8_t* tb = p.qk_bias + (static_cast<int64_t>(p.Hq) * prow + static_cast<int64_t>(hq) * ntile * 128 +
                                        tile * 128) * 32;
             uint8_t* row = tb + (rl >> 3) * 256 + (rl & 7) * 16;
-            *reinterpret_cast<uint4*>(row) = make_uint4(w0, w1, 0u, 0u);
-            *reinterpret_cast<uint4*>(row + 128) = make_uint4(0u, 0u, 0u, 0u);
+            if (SAGE_IN_BOUNDS(static_cast<uint64_t>(row + 144 - p.qk_bias) <= p.lim.qk_bias, p.err, nullptr)) {
+              *reinterpret_cast<uint4*>(row) = make_uint4(w0, w1, 0u, 0u);
+              *reinterpret_cast<uint4*>(row + 128) = make_uint4(0u, 0u, 0u, 0u);
+            }
           }
         }
       }
@@ -525,7 +547,9 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(QuantParams p) {
       const uint32_t sb = block_scale_byte(a);
       const float s = e4m3_to_f32(sb);
       const uint32_t w = encode8(x, s);
-      *reinterpret_cast<uint32_t*>(dst + static_cast<size_t>(rl) * (D / 2) + c * 4) = w;
+      if (SAGE_IN_BOUNDS(static_cast<uint64_t>(row0 + rl) * (D / 2) + c * 4 + 4 <= (job == 0 ? p.lim.q_fp4 : p.lim.k_fp4),
+                         p.err, nullptr))
+        *reinterpret_cast<uint32_t*>(dst + static_cast<size_t>(rl) * (D / 2) + c * 4) = w;
       if ((c & 1) == 0) {
         const int col = c * 8;
         sfbuf[(col / 64) * 512 + (rl % 32) * 16 + (rl / 32) * 4 + (col % 64) / 16] = static_cast<uint8_t>(sb);
@@ -533,8 +557,9 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(QuantParams p) {
     }
     __syncthreads();
     uint8_t* sf_out = (job == 0 ? p.q_sf : p.k_sf) + T * kSfBytesQK;
-    for (int i = t; i < kSfBytesQK / 16; i += kThreads)
-      reinterpret_cast<uint4*>(sf_out)[i] = reinterpret_cast<const uint4*>(sfbuf)[i];
+    if (SAGE_IN_BOUNDS(static_cast<uint64_t>(T + 1) * kSfBytesQK <= (job == 0 ? p.lim.q_sf : p.lim.k_sf), p.err, nullptr))
+      for (int i = t; i < kSfBytesQK / 16; i += kThreads)
+        reinterpret_cast<uint4*>(sf_out)[i] = reinterpret_cast<const uint4*>(sfbuf)[i];
   } else {
     // ---- V^T: tokens become the contiguous (contraction) dimension ----
     uint8_t* vtile = smem;                                // 128 x kVRowBytes
@@ -548,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(QuantParams p) {
   #pragma unroll
       for (int it = 0; it < kIter; ++it) {
         const int rl = rl0 + it * kRowStep;
-        raw[it] = rl < rows ? ld_nc_16(row_ptr(p.v, p.sv, b, h, tok0 + rl) + c * 16) : make_uint4(0, 0, 0, 0);
+        raw[it] = rl < rows ? ld_row16(p.v, p.sv, b, h, tok0 + rl, c, p.lim.v_el, p.err) : make_uint4(0, 0, 0, 0);
       }
   #pragma unroll
       for (int it = 0; it < kIter; ++it)
@@ -582,13 +607,15 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(QuantParams p) {
     }
     __syncthreads();
     uint8_t* vt = p.vt_fp4 + T * (D * 64);
-    for (int gi = t; gi < D * 4; gi += kThreads) {
-      const int d = gi / 4, k = gi % 4;
-      *reinterpret_cast<uint4*>(vt + d * 64 + k * 16) = *reinterpret_cast<const uint4*>(cbuf + d * kCodeRow + k * 16);
-    }
+    if (SAGE_IN_BOUNDS(static_cast<uint64_t>(T + 1) * (D * 64) <= p.lim.vt_fp4, p.err, nullptr))
+      for (int gi = t; gi < D * 4; gi += kThreads) {
+        const int d = gi / 4, k = gi % 4;
+        *reinterpret_cast<uint4*>(vt + d * 64 + k * 16) = *reinterpret_cast<const uint4*>(cbuf + d * kCodeRow + k * 16);
+      }
     uint8_t* sf_out = p.vt_sf + T * 1024;
-    for (int i = t; i < 1024 / 16; i += kThreads)
-      reinterpret_cast<uint4*>(sf_out)[i] = reinterpret_cast<const uint4*>(sfbuf)[i];
+    if (SAGE_IN_BOUNDS(static_cast<uint64_t>(T + 1) * 1024 <= p.lim.vt_sf, p.err, nullptr))
+      for (int i = t; i < 1024 / 16; i += kThreads)
+        reinterpret_cast<uint4*>(sf_out)[i] = reinterpret_cast<const uint4*>(sfbuf)[i];
   }
 }
 
@@ -643,7 +670,8 @@ __global__ void __launch_bounds__(kThreads, 4) quant8_kernel(QuantParams p) {
 #pragma unroll
     for (int it = 0; it < kIter; ++it) {
       const int rl = rl0 + it * kRowStep;
-      raw[it] = rl < rows ? ld_nc_16(row_ptr(src, st, b, h, tok0 + rl) + c * 16) : make_uint4(0, 0, 0, 0);
+      raw[it] = rl < rows ? ld_row16(src, st, b, h, tok0 + rl, c, job == 0 ? p.lim.q_el : p.lim.k_el, p.err)
+                          : make_uint4(0, 0, 0, 0);
     }
     auto values = [&](int it, float (&x)[8]) {
       unpack8(raw[it], p.dtype, x);
@@ -663,7 +691,8 @@ __global__ void __launch_bounds__(kThreads, 4) quant8_kernel(QuantParams p) {
     a = block_max(a, redw);
     const float s = __fdiv_rn(a, 127.0f);
     const double cs = s > 0.0f ? recip_d(s) : 0.0;  // x / s = div_by(x, cs)
-    if (t == 0) reinterpret_cast<float*>(job == 0 ? p.q_sf : p.k_sf)[T] = s;
+    if (t == 0 && SAGE_IN_BOUNDS(static_cast<uint64_t>(T + 1) * 4 <= (job == 0 ? p.lim.q_sf : p.lim.k_sf), p.err, nullptr))
+      reinterpret_cast<float*>(job == 0 ? p.q_sf : p.k_sf)[T] = s;
     uint8_t* dst = (job == 0 ? p.q_fp4 : p.k_fp4) + row0 * D;
 #pragma unroll
     for (int it = 0; it < kIter; ++it) {
@@ -677,7 +706,9 @@ __global__ void __launch_bounds__(kThreads, 4) quant8_kernel(QuantParams p) {
           w[e >> 2] |= (static_cast<uint32_t>(static_cast<int>(r)) & 0xFFu) << (8 * (e & 3));
         }
       }
-      *reinterpret_cast<uint2*>(dst + static_cast<size_t>(rl0 + it * kRowStep) * D + c * 8) = make_uint2(w[0], w[1]);
+      if (SAGE_IN_BOUNDS(static_cast<uint64_t>(row0 + rl0 + it * kRowStep) * D + c * 8 + 8 <=
+                             (job == 0 ? p.lim.q_fp4 : p.lim.k_fp4), p.err, nullptr))
+        *reinterpret_cast<uint2*>(dst + static_cast<size_t>(rl0 + it * kRowStep) * D + c * 8) = make_uint2(w[0], w[1]);
     }
   } else {
   // ---- V^T: E4M3 with one scale per channel ----
@@ -689,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant8_kernel(QuantParams p) {
 #pragma unroll
     for (int it = 0; it < kIter; ++it) {
       const int rl = rl0 + it * kRowStep;
-      raw[it] = rl < rows ? ld_nc_16(row_ptr(p.v, p.sv, b, h, tok0 + rl) + c * 16) : make_uint4(0, 0, 0, 0);
+      raw[it] = rl < rows ? ld_row16(p.v, p.sv, b, h, tok0 + rl, c, p.lim.v_el, p.err) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int it = 0; it < kIter; ++it)
@@ -727,7 +758,8 @@ __global__ void __launch_bounds__(kThreads, 4) quant8_kernel(QuantParams p) {
   uint8_t* vt = p.vt_fp4 + T * (D * 128);
   for (int gi = t; gi < D * 8; gi += kThreads) {
     const int d = gi / 8, k = gi % 8;
-    *reinterpret_cast<uint4*>(vt + d * 128 + k * 16) = *reinterpret_cast<const uint4*>(cbuf + d * kCodeRow + k * 16);
+    if (SAGE_IN_BOUNDS(static_cast<uint64_t>(T) * (D * 128) + d * 128 + k * 16 + 16 <= p.lim.vt_fp4, p.err, nullptr))
+      *reinterpret_cast<uint4*>(vt + d * 128 + k * 16) = *reinterpret_cast<const uint4*>(cbuf + d * kCodeRow + k * 16);
   }
   }
 }

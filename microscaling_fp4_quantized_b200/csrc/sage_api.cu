@@ -198,6 +198,46 @@ sage_fp4_problem_sizes_t sizes_of(const Prob& p) {
   return z;
 }
 
+// Elements of a caller tensor the problem can reach: the largest offset of a (sequence,
+// head, token) row through the strides, plus the row's D channels (0 when empty).
+uint64_t extent_el(const int64_t* st, int64_t B, int64_t H, int64_t tokens, bool packed, int64_t D) {
+  if (B <= 0 || H <= 0 || tokens <= 0) return 0;
+  const int64_t last = (packed ? 0 : (B - 1) * st[0]) + (H - 1) * st[1] + (tokens - 1) * st[2];
+  return static_cast<uint64_t>(last + D);
+}
+
+// The extents every kernel of the problem may touch (see sage::Limits).
+sage::Limits limits_of(const Prob& p) {
+  sage::Limits l;
+  std::memset(&l, 0, sizeof(l));
+  if (p.empty) return l;
+  const sage_fp4_problem_sizes_t z = sizes_of(p);
+  const int64_t B = p.u.B, Hq = p.u.Hq, Hkv = p.u.Hkv, D = p.u.D, ns = p.nsplit;
+  const int64_t tq = p.packed ? p.u.total_q : p.u.Nq, tk = p.packed ? p.u.total_k : p.u.Nk;
+  l.q_el = extent_el(p.u.q_stride, B, Hq, tq, p.packed, D);
+  l.k_el = extent_el(p.u.k_stride, B, Hkv, tk, p.packed, D);
+  l.v_el = extent_el(p.u.v_stride, B, Hkv, tk, p.packed, D);
+  l.o_el = extent_el(p.u.o_stride, B, Hq, tq, p.packed, D);
+  l.q_fp4 = z.q_fp4;
+  l.k_fp4 = z.k_fp4;
+  l.vt_fp4 = z.vt_fp4;
+  l.q_sf = z.q_sf;
+  l.k_sf = z.k_sf;
+  l.vt_sf = z.vt_sf;
+  l.qk_bias = z.qk_bias;
+  l.k_mean_el = z.k_mean / 4;
+  l.q_mean_el = z.q_mean / 4;
+  l.amax_el = z.amax / 4;
+  l.stat_el = static_cast<uint64_t>(B * Hkv * ns * D);
+  l.qstat_el = static_cast<uint64_t>(B * Hq * ns * D);
+  l.qamax_el = static_cast<uint64_t>(B * Hq * ns);
+  l.vamax_el = static_cast<uint64_t>(B * Hkv * ns);
+  l.rows_q = static_cast<uint64_t>(Hq * p.rows_q);
+  l.rows_k = static_cast<uint64_t>(Hkv * p.rows_k);
+  l.rows_v = static_cast<uint64_t>(Hkv * p.rows_k / 128 * D);
+  return l;
+}
+
 // Carve a workspace (256-byte aligned) into the quantized bundle followed by the scratch.
 void carve(const Prob& p, void* base, sage_fp4_quantized_t* qz, void** scratch) {
   const sage_fp4_problem_sizes_t z = sizes_of(p);
@@ -317,6 +357,7 @@ sage_status_t run_quantize(const Prob& p, const void* q, const void* k, const vo
     k_.bad_out = reinterpret_cast<uint32_t*>(qz.seq + 2 * (p.u.B + 1));
   }
   k_.err = err;
+  k_.lim = limits_of(p);
   if (p.b8) return cuda_status(sage::launch_quantize8(k_, sage::QuantLaunch{p.tiles_q, p.tiles_k}, stream));
   return cuda_status(sage::launch_quantize(k_, sage::QuantLaunch{p.tiles_q, p.tiles_k}, stream));
 }
@@ -380,6 +421,8 @@ sage_status_t run_attention(const Prob& p, const sage_fp4_quantized_t& qz, void*
   a.Hkv = p.u.Hkv;
   a.group = p.u.Hq / p.u.Hkv;
   a.seq = seq_map(p, qz);
+  a.lim = limits_of(p);
+  if (a.debug_flags & sage::kDebugNoOutput) a.lim.o_el = 0;
   a.amax = p.gs ? qz.amax : nullptr;
   a.qk_bias = p.sq ? qz.qk_bias : nullptr;
   if (p.b8) {
@@ -423,6 +466,7 @@ const char* sage_status_string(sage_status_t status) {
     case SAGE_ERR_UNSUPPORTED: return "SAGE_ERR_UNSUPPORTED";
     case SAGE_ERR_CUDA: return "SAGE_ERR_CUDA";
     case SAGE_ERR_TIMEOUT: return "SAGE_ERR_TIMEOUT";
+    case SAGE_ERR_BOUNDS: return "SAGE_ERR_BOUNDS";
   }
   return "SAGE_ERR_UNKNOWN";
 }
@@ -621,15 +665,28 @@ sage_status_t sage_fp4_get_device_error(uint32_t* word, void* stream) {
   if (cudaStreamSynchronize(s) != cudaSuccess) return SAGE_ERR_CUDA;
   *word = host;
   if (host == 0) return SAGE_OK;
-  return (host & sage::kDevErrTimeout) ? SAGE_ERR_TIMEOUT : SAGE_ERR_INVALID_ARG;
+  if (host & sage::kDevErrTimeout) return SAGE_ERR_TIMEOUT;
+  if (host & sage::kDevErrBounds) return SAGE_ERR_BOUNDS;
+  return SAGE_ERR_INVALID_ARG;
 }
 
 const char* sage_fp4_last_cuda_error(void) { return g_last_error; }
 
 sage_status_t sage_fp4_set_debug_flags(uint32_t flags) {
-  if (flags & ~1u) return SAGE_ERR_INVALID_ARG;
+  if (flags & ~3u) return SAGE_ERR_INVALID_ARG;
+#ifndef SAGE_CHECKS
+  if (flags & sage::kDebugNoOutput) return SAGE_ERR_UNSUPPORTED;  // only the bounds-checked build has it
+#endif
   g_debug_flags.store(flags);
   return SAGE_OK;
+}
+
+int sage_fp4_bounds_checked(void) {
+#ifdef SAGE_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
 }
 
 sage_status_t sage_fp4_mma_rate(int n, int iters, int ctas, void* stream) {

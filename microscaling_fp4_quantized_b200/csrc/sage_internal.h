@@ -11,7 +11,35 @@ namespace sage {
 enum : int { kDtypeBF16 = 0, kDtypeF16 = 1 };
 
 // Bits of the device error word.
-enum : uint32_t { kDevErrTimeout = 1u, kDevErrSeqlens = 2u };
+enum : uint32_t { kDevErrTimeout = 1u, kDevErrSeqlens = 2u, kDevErrBounds = 4u };
+
+// Extents the kernels may touch, derived on the host from the problem: elements of the
+// caller's q, k, v and out reachable through the strides, bytes of each quantized
+// buffer, elements of the statistics buffers, and rows of the TMA maps. The bounds-checked
+// build (compiled with SAGE_CHECKS) tests every computed global index against them before
+// the access; a failed check sets kDevErrBounds in the device error word, raises the CTA's
+// abort flag where the kernel has one, and skips the access. Without SAGE_CHECKS the
+// checks compile to nothing and these fields are unused.
+struct Limits {
+  uint64_t q_el, k_el, v_el, o_el;
+  uint64_t q_fp4, k_fp4, vt_fp4, q_sf, k_sf, vt_sf, qk_bias;
+  uint64_t k_mean_el, q_mean_el, amax_el, stat_el, qstat_el, qamax_el, vamax_el;
+  uint64_t rows_q, rows_k, rows_v;
+};
+
+#ifdef SAGE_CHECKS
+// True when `cond` holds; otherwise records a bounds failure (and raises *abort_flag when
+// it is not null) and returns false so that the caller skips the access.
+__device__ __forceinline__ bool sage_in_bounds(bool cond, uint32_t* err, volatile uint32_t* abort_flag) {
+  if (cond) return true;
+  atomicOr(err, kDevErrBounds);
+  if (abort_flag != nullptr) *abort_flag = 1u;
+  return false;
+}
+#define SAGE_IN_BOUNDS(cond, err, abort_flag) ::sage::sage_in_bounds((cond), (err), (abort_flag))
+#else
+#define SAGE_IN_BOUNDS(cond, err, abort_flag) true
+#endif
 
 // Second-level scale modes (one FP32 factor per tensor or per (sequence, head)).
 enum : int { kGscaleNone = 0, kGscaleTensor = 1, kGscaleHead = 2 };
@@ -132,6 +160,7 @@ struct QuantParams {
   int32_t* pad_k_out;
   uint32_t* bad_out;
   uint32_t* err;
+  Limits lim;
 };
 
 struct AttnParams {
@@ -159,9 +188,13 @@ struct AttnParams {
   uint64_t timeout_ns;  // bound on every wait
   uint32_t debug_flags; // kDebugNoLoads: the producer issues no copies (test of the error path)
   int tiles_q;          // query tiles of the longest sequence (work items: B * Hq * tiles_q)
+  Limits lim;
 };
 
-enum : uint32_t { kDebugNoLoads = 1u };
+// Test switches: kDebugNoLoads, the attention kernel's copy warps issue no loads (every
+// bounded wait then runs out); kDebugNoOutput (bounds-checked build only), the output
+// extent is taken as 0, so every output store fails its check and is skipped.
+enum : uint32_t { kDebugNoLoads = 1u, kDebugNoOutput = 2u };
 
 struct TensorMaps {
   CUtensorMap q, k, v;

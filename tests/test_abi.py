@@ -126,3 +126,22 @@ def test_8bit_problem_sizes_and_refusals(L):
         with pytest.raises(sage.SageError) as e:
             sage.problem_sizes(_dense_pr(sage, precision="8bit", **bad))
         assert e.value.status == sage.SAGE_ERR_UNSUPPORTED
+
+
+def test_bounds_checked_build_loads_and_reports_itself():
+    """The bounds-checked variant exports the same entry points and says it is checked;
+    the regular build says it is not, and refuses the checked build's test switch."""
+    import ctypes
+    from microscaling_fp4_quantized_b200 import build as b
+    path = b.build(checks=True)
+    C = ctypes.CDLL(path)
+    for name in _declared():
+        assert hasattr(C, name), name
+    assert C.sage_fp4_bounds_checked() == 1
+    R = ctypes.CDLL(b.build())
+    assert R.sage_fp4_bounds_checked() == 0
+    R.sage_fp4_set_debug_flags.argtypes = [ctypes.c_uint32]
+    C.sage_fp4_set_debug_flags.argtypes = [ctypes.c_uint32]
+    assert R.sage_fp4_set_debug_flags(2) == 2       # SAGE_ERR_UNSUPPORTED
+    assert C.sage_fp4_set_debug_flags(2) == 0 and C.sage_fp4_set_debug_flags(0) == 0
+    assert R.sage_fp4_set_debug_flags(4) == 1       # SAGE_ERR_INVALID_ARG

@@ -59,5 +59,10 @@ def test_bounded_wait_reports_timeout_and_context_survives(sage, oracle_mod, wl)
 
 def test_debug_flags_reject_unknown_bits(sage):
     with pytest.raises(sage.SageError) as e:
-        sage.set_debug_flags(2)
+        sage.set_debug_flags(4)
     assert e.value.status == sage.SAGE_ERR_INVALID_ARG
+    if not sage.lib().sage_fp4_bounds_checked():
+        # the output-extent switch exists in the bounds-checked build only
+        with pytest.raises(sage.SageError) as e:
+            sage.set_debug_flags(2)
+        assert e.value.status == sage.SAGE_ERR_UNSUPPORTED
