@@ -1,7 +1,8 @@
 """Host logic of the multi-GPU bench path on CPU: two gloo ranks on 127.0.0.1.
 
-Each rank runs its own copy of the workload (independent problems, weak scaling, no
-data-path collective); the only cross-rank step is the MAX reduction of device times.
+Each rank holds and computes its own slice of the (batch, head) pairs of one problem (the
+workload's shape per rank, weak scaling, no data-path collective); the only cross-rank step
+is the MAX reduction of device times.
 """
 import json
 import os

@@ -75,3 +75,45 @@ def test_gather_reassembles_in_pair_order(n_pairs):
     for _ in range(2):
         rank, full = q.get(timeout=10)
         assert full == want, rank
+
+
+def _attn_worker(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import numpy as np
+    import oracle
+    from microscaling_fp4_quantized_b200 import shard as sh
+    n_pairs, N, D = 5, 96, 64
+    g = np.random.default_rng(7)                       # every rank draws the same whole problem
+    qq, kk, vv = (g.standard_normal((n_pairs, N, D)) for _ in range(3))
+    lo, hi = sh.head_slice(n_pairs, world, rank)
+    o_r, _ = oracle.attention(qq[lo:hi], kk[lo:hi], vv[lo:hi], True, D ** -0.5)
+    full = sh.gather_heads(torch.from_numpy(np.ascontiguousarray(o_r)), n_pairs)
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((rank, full.numpy()))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sliced_forward_equals_whole_problem(world):
+    """Each rank runs the (oracle) FP4 forward on its slice of 5 pairs and gathers: every
+    rank must hold exactly the whole problem's result, pair order kept."""
+    import numpy as np
+    import oracle
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_attn_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=180) for _ in range(world)]
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    g = np.random.default_rng(7)
+    qq, kk, vv = (g.standard_normal((5, 96, 64)) for _ in range(3))
+    want, _ = oracle.attention(qq, kk, vv, True, 64 ** -0.5)
+    for rank, full in got:
+        assert full.shape == want.shape, rank
+        assert np.array_equal(full, want), rank
