@@ -423,8 +423,9 @@ def time_e2e(sage, wl, q, k, v, dev, stream, steps, dist, world, precision="fp4"
             "serial": {"value": job_value(wl.ops, world, ms_s), "ms_per_step": ms_s}}
 
 
-# Kernels per step: K statistics, K mean, Q/K quantization, V^T quantization, attention.
-LAUNCHES_PER_STEP = 5
+# Kernels per step: quantizer pass A (K statistics, Q, V^T), K mean, quantizer pass B (K),
+# attention.
+LAUNCHES_PER_STEP = 4
 
 
 def time_general(sage, gw, dev, stream, warmup, steps, inputs=None):
