@@ -30,10 +30,10 @@ __device__ __forceinline__ bool try_wait_for(uint32_t bar, uint32_t parity, uint
 // Bounded wait: true when the phase with `parity` has completed, false on abort/timeout.
 // sleep_ns != 0 lets the thread stay suspended in each probe for up to that long; the
 // abort flag and the clock are read after every probe whose index & check_mask is 0.
-// Measured on the FP4 attention kernel: its non-causal instances run fastest with
-// suspended probes and a check after each, the causal ones with plain probes and a
-// check every 32nd (per-tile times 1110 vs 1225 ns on long non-causal rows, 1413 vs
-// 1785 ns on causal ones).
+// Measured on the FP4 attention kernel: every role waits fastest with plain probes and a
+// check every 32nd (1158 against 1100 TFLOP/s with 500 ns suspended probes on long
+// non-causal rows, 822 against 781 on causal ones); suspending only the copy and MMA
+// warps lost on causal rows.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& c, uint32_t sleep_ns = 0u,
                                          uint32_t check_mask = 0u) {
   if (try_wait_for(bar, parity, sleep_ns)) return true;

@@ -1,8 +1,7 @@
 // FP4 attention forward (sm_100a): the non-causal instances of the kernel template in
 // attn_fp4_kernel.cuh, the launch dispatch, and the S = Q^ K^^T check kernel. The causal
-// instances live in their own translation unit (attn_fp4_causal.cu): the kernel's speed
-// depends on its instruction fetch, and the measured best wait policy differs between
-// the two (see wait_bar).
+// instances live in their own translation unit (attn_fp4_causal.cu), which keeps the two
+// sets of instances compiling in parallel.
 #include "attn_fp4_kernel.cuh"
 
 namespace sage {

@@ -141,6 +141,7 @@ struct Layout {
   static constexpr int kNumBars = 40;
   static constexpr int off_misc = off_bar + kNumBars * 8;    // tmem base, abort flag, drain flags
   static constexpr int kBytes = off_misc + 32;
+  static_assert(kBytes + 1024 <= 227 * 1024, "shared memory above the per-CTA limit");
 };
 
 // Barrier indices.
