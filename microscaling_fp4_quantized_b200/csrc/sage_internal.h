@@ -209,9 +209,6 @@ cudaError_t launch_quantize8(const QuantParams& p, const QuantLaunch& l, cudaStr
 cudaError_t launch_attention(const TensorMaps& maps, const AttnParams& p, int tiles_q, cudaStream_t stream);
 cudaError_t launch_qk_scores(const TensorMaps& maps, const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_attention8(const TensorMaps& maps, const AttnParams& p, int tiles_q, cudaStream_t stream);
-// Up to this many query tiles per (sequence, head), launch_attention runs one CTA per SM
-// over all work items instead of one CTA per item.
-constexpr int kShortTiles = 8;
 // Tensor-core rate probe (mma_rate.cu): `ctas` CTAs, each issuing `iters` block-scaled FP4
 // products of M = 128, N = n, K = 64.
 cudaError_t launch_mma_rate(int n, int iters, int ctas, uint32_t* err, uint64_t timeout_ns, cudaStream_t stream);
