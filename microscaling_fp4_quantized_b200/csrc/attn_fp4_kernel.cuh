@@ -195,21 +195,22 @@ struct WorkItem {
   bool valid;        // the sequence has this query tile
 };
 
-// Item w of the list: query-tile index fastest (consecutive items share their key/value
-// head, which keeps its K^ / V^T tiles in L2), causal tiles longest first within a head.
-// The k-th work item of this CTA, or -1 past the end of the list. Round k hands items
-// kG .. kG + G - 1 to the G CTAs. Causal items shrink along the list (heaviest first, see
-// decode_item), so odd rounds go in reverse CTA order and every CTA ends with about the
-// same work (measured on the causal LLM workload: 1025 against 924 TFLOP/s in plain
-// order). Non-causal items are all alike and keep the plain order, which measured faster
-// for them.
+// The walk over the work items: round k hands items kG .. kG + G - 1 to the G CTAs.
+// Causal items shrink along the list (heaviest first, see decode_item), so odd rounds go
+// in reverse CTA order and every CTA ends with about the same work (measured on the causal
+// LLM workload: 1033 against 924 TFLOP/s in plain order). Non-causal items are all alike
+// and keep the plain order, which measured faster for them. next_item gets round k + 1 and
+// the item of round k; the walk ends at an item >= the item count.
 template <bool CAUSAL>
-__device__ __forceinline__ int item_of(int k, int n_items) {
+__device__ __forceinline__ int next_item(int k1, int w) {
   const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
-  const int w = k * G + ((CAUSAL && (k & 1)) ? G - 1 - c : c);
-  return w < n_items ? w : -1;
+  if (!CAUSAL) return w + G;
+  return k1 * G + ((k1 & 1) ? G - 1 - c : c);
 }
 
+// Item w of the list. Non-causal: query-tile index fastest (consecutive items share their
+// key/value head, which keeps its K^ / V^T tiles in L2). Causal: heaviest first over all
+// (sequence, head) pairs.
 template <bool GENERAL, bool CAUSAL>
 __device__ __forceinline__ void decode_item(const AttnParams& p, int w, WorkItem& it) {
   const int per_head = p.tiles_q;
@@ -349,7 +350,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (lane == 0 && !(p.debug_flags & kDebugNoLoads)) {
       int gt = 0, qi = 0;
       bool ok = true;
-      for (int k = 0, w; ok && (w = item_of<CAUSAL>(k, n_items)) >= 0; ++k) {
+      for (int k = 0, w = blockIdx.x; ok && w < n_items; ++k, w = next_item<CAUSAL>(k, w)) {
         WorkItem it;
         decode_item<GENERAL, CAUSAL>(p, w, it);
         if (!it.valid || it.nt == 0) continue;
@@ -397,7 +398,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (lane == 0 && !(p.debug_flags & kDebugNoLoads)) {
       int gt = 0;
       bool ok = true;
-      for (int k = 0, w; ok && (w = item_of<CAUSAL>(k, n_items)) >= 0; ++k) {
+      for (int k = 0, w = blockIdx.x; ok && w < n_items; ++k, w = next_item<CAUSAL>(k, w)) {
         WorkItem it;
         decode_item<GENERAL, CAUSAL>(p, w, it);
         if (!it.valid) continue;
@@ -429,7 +430,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       constexpr int kc_qk = D / 64;
       int gt = 0, qi = 0;
       bool ok = true;
-      for (int k = 0, w; ok && (w = item_of<CAUSAL>(k, n_items)) >= 0; ++k) {
+      for (int k = 0, w = blockIdx.x; ok && w < n_items; ++k, w = next_item<CAUSAL>(k, w)) {
         WorkItem it;
         decode_item<GENERAL, CAUSAL>(p, w, it);
         if (!it.valid || it.nt == 0) continue;
@@ -477,7 +478,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       constexpr uint32_t idesc_pv = make_idesc_fp4(D);
       int gt = 0;
       bool ok = true;
-      for (int k = 0, w; ok && (w = item_of<CAUSAL>(k, n_items)) >= 0; ++k) {
+      for (int k = 0, w = blockIdx.x; ok && w < n_items; ++k, w = next_item<CAUSAL>(k, w)) {
         WorkItem it;
         decode_item<GENERAL, CAUSAL>(p, w, it);
         if (!it.valid) continue;
@@ -518,7 +519,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     int gt = 0, itc = 0;
     bool ok = true;
-    for (int k = 0, wi; ok && (wi = item_of<CAUSAL>(k, n_items)) >= 0; ++k) {
+    for (int k = 0, wi = blockIdx.x; ok && wi < n_items; ++k, wi = next_item<CAUSAL>(k, wi)) {
       WorkItem it;
       decode_item<GENERAL, CAUSAL>(p, wi, it);
       if (!it.valid) continue;
@@ -610,7 +611,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint8_t* sfrow = smem + L::off_sfp + sw * L::kSfPBytes + (r % 32) * 16 + (r / 32) * 4;
     int gt = 0, itc = 0;
     bool ok = true;
-    for (int k = 0, wi; ok && (wi = item_of<CAUSAL>(k, n_items)) >= 0; ++k) {
+    for (int k = 0, wi = blockIdx.x; ok && wi < n_items; ++k, wi = next_item<CAUSAL>(k, wi)) {
       WorkItem it;
       decode_item<GENERAL, CAUSAL>(p, wi, it);
       if (!it.valid) continue;

@@ -155,8 +155,8 @@ def test_attn_alternating_tile_maxima(sage, oracle_mod, causal):
 
 
 def test_attn_short_dense_many_items_per_cta(sage, oracle_mod):
-    """Square dense non-causal D = 128 with at most 8 query tiles takes the persistent
-    kernel: 2 x 96 heads x 8 query tiles = 1536 work items over one CTA per SM (about ten
-    items each, consecutive items of a CTA in different heads), with a ragged last tile."""
+    """Square dense non-causal D = 128, short rows: 2 x 96 heads x 8 query tiles = 1536
+    work items over one CTA per SM (about ten items each, consecutive items of a CTA in
+    different heads), with a ragged last tile."""
     wl = workloads.custom(2, 96, 1000, 128, seed=62)
     _check(sage, oracle_mod, wl, heads=[0, 95, 191], rows_per_head=40)

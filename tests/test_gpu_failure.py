@@ -23,9 +23,10 @@ def sage():
     return s
 
 
-# A causal problem (one CTA per query tile) and a short dense non-causal D = 128 problem
-# with many (sequence, head, query tile) items per CTA (the persistent path, whose abort
-# and drain code differs: drains of its last Q/K/V loads and of both MMA issuers).
+# A causal problem with fewer work items than SMs (one item per CTA) and a short dense
+# non-causal D = 128 problem with many (sequence, head, query tile) items per CTA, so that
+# the abort reaches CTAs in the middle of their walk (drains of the last Q/K/V loads and
+# of both MMA issuers with several items behind them).
 CASES = [workloads.custom(1, 2, 384, 128, causal=True, seed=61),
          workloads.custom(8, 32, 1024, 128, causal=False, seed=62)]
 
