@@ -160,3 +160,15 @@ def test_attn_short_dense_many_items_per_cta(sage, oracle_mod):
     different heads), with a ragged last tile."""
     wl = workloads.custom(2, 96, 1000, 128, seed=62)
     _check(sage, oracle_mod, wl, heads=[0, 95, 191], rows_per_head=40)
+
+
+@pytest.mark.parametrize("D", [128, 64])
+def test_attn_causal_walk_partial_reversed_round(sage, oracle_mod, D):
+    """Causal rows walk their work items heaviest first over all (sequence, head) pairs,
+    odd rounds in reverse CTA order. 2 x 104 heads x 8 query tiles = 1664 items over the
+    148 CTAs of a B200 is 11 full rounds and a partial 12th, which is an odd (reversed)
+    round: it holds the lightest items, query tile 0 of pairs 172-207, taken by the last
+    CTAs. Every row of the pairs on either side of that boundary is checked, and the last
+    query tile (the ragged one) of the first pair."""
+    wl = workloads.custom(2, 104, 1000, D, causal=True, seed=63)
+    _check(sage, oracle_mod, wl, heads=[0, 171, 172, 207])
