@@ -8,11 +8,12 @@
 // diag(l)^-1 after the last key tile (reply to Q2), and the two-level P~ quantization
 // (per-row factor s1 = rowmax(P~)/(448*6) per key tile, then 16-element E4M3 scales).
 //
-// Work items are (sequence, query head, 128-query tile); key tiles are 128 wide. CTA c
-// takes items c, c + gridDim.x, ... (one item per CTA when the grid covers them all, a
-// persistent walk over many items when it is one CTA per SM); every role derives the
-// same list, and barrier phases follow CTA-wide counts of key tiles and items, so the
-// next item's copies and products start while the current item finishes. Sequences may
+// Work items are (sequence, query head, 128-query tile); key tiles are 128 wide. The grid
+// is at most one CTA per SM, and each CTA walks its share of the item list (next_item:
+// plain order for non-causal problems, heaviest first and alternating rounds for causal
+// ones); every role derives the same list, and barrier phases follow CTA-wide counts of
+// key tiles and items, so the next item's copies and products start while the current
+// item finishes. Sequences may
 // be packed with different lengths, query heads may share key/value heads (head h reads
 // key/value head h / (Hq / Hkv)), and the causal mask keeps key j <= i + (len_k - len_q).
 //
@@ -776,7 +777,7 @@ static int attn_smem_bytes() {
   return need > 116 * 1024 ? need : 116 * 1024;
 }
 
-// Grid: one CTA per work item, or (persistent) at most `max_ctas` CTAs walking the list.
+// Grid: the smaller of the item count and `max_ctas`, every CTA walking its share.
 template <int D, bool CAUSAL, int MODE>
 static cudaError_t launch_attn_t(const TensorMaps& m, const AttnParams& p, int tiles_q, int max_ctas,
                                  cudaStream_t stream) {

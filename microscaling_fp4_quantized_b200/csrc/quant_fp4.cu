@@ -822,14 +822,14 @@ __global__ void __launch_bounds__(kThreads, pass_min_blocks<KINDS>()) quant_pass
 }
 
 // ------------------------------------------------------------- 8-bit path ----
-// Two launches, split like quant_kernel. VJOB = false, grid (2 * tiles, Hq, B),
+// Two launches: VJOB = false, grid (2 * tiles, Hq, B),
 // x = 2 * tile + job: jobs 0 and 1 turn a 128-row tile of Q or K - mean into symmetric
 // INT8 with one scale s = fp32(absmax / 127) for the tile and codes
 // clamp(RNE(fp32(x / s)), -127, 127). VJOB = true, grid (key tiles, Hkv, B): a 128-token
 // tile of V becomes E4M3 codes fp32(v / s_d) with the channel scales of the finalize
 // pass, transposed (tokens contiguous) and stored tile-major [key tiles, D, 128].
-// Bounded to 4 CTAs per SM like quant_kernel (0.48 -> 0.46 ms for the long workload's
-// 8-bit quantization, identical output bytes).
+// Only the V^T launch needs the large shared-memory tile. Bounded to 4 CTAs per SM
+// (0.48 -> 0.46 ms for the long workload's 8-bit quantization, identical output bytes).
 template <int D, bool VJOB>
 __global__ void __launch_bounds__(kThreads, 4) quant8_kernel(QuantParams p) {
   constexpr int CPR = D / 8;
