@@ -63,6 +63,25 @@ def test_quant_without_smoothing(sage, oracle_mod):
     _compare_quant(sage, oracle_mod, q, k, v, smooth_k=False)
 
 
+@pytest.mark.parametrize("D", [128, 64])
+def test_quant_inputs_off_32_byte_boundary(sage, oracle_mod, D):
+    """Inputs 16 bytes past a 32-byte boundary (the API asks for 16): the quantizer then
+    reads each 16-element block as two 16-byte pieces instead of one 32-byte piece. Codes,
+    scales and the K mean must be the same bit for bit."""
+    wl = workloads.custom(1, 2, 300, D, seed=16)
+    q, k, v = workloads.make_inputs(wl, device="cuda")
+
+    def shifted(t):
+        buf = torch.empty(t.numel() + 8, dtype=t.dtype, device=t.device)
+        s = buf[8:].view(t.shape)
+        s.copy_(t)
+        return s
+
+    qs, ks, vs = shifted(q), shifted(k), shifted(v)
+    assert qs.data_ptr() % 32 == 16 and ks.data_ptr() % 32 == 16 and vs.data_ptr() % 32 == 16
+    _compare_quant(sage, oracle_mod, qs, ks, vs)
+
+
 def _edge_tensor(D, N, dtype):
     """Blocks built to land on E2M1 and E4M3 rounding ties, signed zeros, saturation,
     subnormal scales and all-zero blocks."""
