@@ -193,8 +193,9 @@ sage_status_t sage_fp4_attn_quantized(const sage_fp4_problem_t* problem, const s
 
 /*
  * The whole forward of a general problem with a caller-owned workspace of at least
- * sizes.workspace bytes (256-byte aligned). Dense problems without a second-level scale
- * launch 4 kernels (K statistics, K mean, quantization, attention); packed problems add
+ * sizes.workspace bytes (256-byte aligned). Four kernel launches: quantization pass A
+ * (the statistics, plus Q and V^T when they need no mean or second-level scale), the K
+ * mean and maxima, quantization pass B (K and the rest), attention; packed problems add
  * the sequence-table kernel.
  */
 sage_status_t sage_fp4_attn(const sage_fp4_problem_t* problem, const void* q, const void* k,
@@ -239,7 +240,8 @@ size_t sage_fp4_workspace_bytes(int B, int H, int N, int D);
 
 /*
  * The whole forward (steps 1-4) with a caller-owned workspace of at least
- * sage_fp4_workspace_bytes() bytes (256-byte aligned). Four kernel launches.
+ * sage_fp4_workspace_bytes() bytes (256-byte aligned). Four kernel launches (quantization
+ * pass A, K mean, quantization pass B, attention).
  */
 sage_status_t sage_fp4_attn_fwd_ex(const void* q, const void* k, const void* v, void* out,
                                    sage_dtype_t dtype, int B, int H, int N, int D, int causal,
