@@ -495,7 +495,8 @@ __device__ __forceinline__ float absmax16(const float (&x)[16]) {
 // every lane holds exactly -div_fma(x, s, r) -- and, for x = +-0 or a product that
 // underflows, the zero of the sign opposite to x's, i.e. minus div_fma's copysign result.
 // E2M1 rounding is symmetric too, so the codes come out with every sign bit inverted,
-// which one XOR puts back.
+// which one XOR puts back. (Checked on the CPU for every E4M3 divisor and every finite
+// quotient tried, +-0 and underflowing products included: tests/div_identity.c.)
 template <int O, int N>
 __device__ __forceinline__ uint32_t encode8_neg(const float (&x)[N], float s) {
   if (s == 0.0f) return 0u;

@@ -13,6 +13,12 @@
  * fp32(double(x) * c) equals x / d, with c the kernel's double reciprocal (the binary32
  * reciprocal refined by two Newton steps in double FMAs, d < 2^-64 scaled by 2^64), for
  * 4000 pseudo-random divisors in [2^-130, 2^21) and every (stride * 641)-th binary32 x.
+ * And the paired-lane form the FP4 quantizer evaluates: with nr = -RN(1/d),
+ * q' = RN(x nr), e = RN(x + q' d) (one FMA), RN(e nr + q') (one FMA) is, bit for bit,
+ * div_fma(x, d) with its sign bit flipped -- for every positive finite E4M3 divisor, both
+ * signs of +-0 and of the 4095 smallest subnormals (whose products underflow), and every
+ * (stride * 67)-th binary32 x of the rest of the finite range whose quotient is finite
+ * (the encoder then flips the E2M1 sign bits back).
  * Prints the number of mismatches of each part; exit status 0 when all are 0. */
 #include <math.h>
 #include <stdint.h>
@@ -42,6 +48,13 @@ static float div_fma(float x, float d, float r) {
   const float q = x * r;
   const float e = fmaf(-q, d, x);
   return copysignf(fmaf(e, r, q), x);
+}
+
+/* The quantizer's negated form: no copysign, every step the negation of div_fma's. */
+static float div_fma_neg(float x, float d, float nr) {
+  const float nq = x * nr;
+  const float e = fmaf(nq, d, x);
+  return fmaf(e, nr, nq);
 }
 
 int main(int argc, char** argv) {
@@ -91,8 +104,24 @@ int main(int argc, char** argv) {
       if (u_of(ref) != u_of(got)) ++badd;
     }
   }
+  long nneg = 0, badneg = 0;
+  for (int b = 1; b <= 0x7E; ++b) {  /* the negated paired-lane form, every E4M3 divisor */
+    const float d = (float)e4m3_value(b), r = 1.0f / d, nr = -r;
+    /* +-0 and the 4095 smallest subnormals one by one, then every (stride * 67)-th x */
+    for (uint32_t u = 0; u < 0x7F800000u; u += (u < 4096u ? 1u : stride * 67u)) {
+      for (int sg = 0; sg < 2; ++sg) {
+        const float x = sg ? -f_of(u) : f_of(u);
+        const float ref = div_fma(x, d, r);
+        if (!isfinite(ref)) continue;  /* |x / d| overflows: never in a block, whose scale */
+                                       /* is at least its absmax / 6 or saturates at 448 */
+        if (u_of(div_fma_neg(x, d, nr)) != (u_of(ref) ^ 0x80000000u)) ++badneg;
+        ++nneg;
+      }
+    }
+  }
   printf("e4m3 divisors: %ld checks, %ld mismatches; d = 6: %ld checks, %ld mismatches; "
          "x / 2688 by a double product: %ld checks, %ld mismatches; x / d by a double product: "
-         "%ld checks, %ld mismatches\n", n, bad, n6, bad6, n2688, bad2688, nd, badd);
-  return (bad == 0 && bad6 == 0 && bad2688 == 0 && badd == 0) ? 0 : 1;
+         "%ld checks, %ld mismatches; negated paired-lane form: %ld checks, %ld mismatches\n",
+         n, bad, n6, bad6, n2688, bad2688, nd, badd, nneg, badneg);
+  return (bad == 0 && bad6 == 0 && bad2688 == 0 && badd == 0 && badneg == 0) ? 0 : 1;
 }

@@ -1,8 +1,10 @@
 """The quantization kernel divides by E4M3 block scales and by 6 with Markstein's
 FMA-corrected quotient instead of a full IEEE division, and the second-level scale
-amax / 2688 is a double-precision product rounded to binary32. This checks, on the CPU,
+amax / 2688 is a double-precision product rounded to binary32. The FP4 quantizer
+evaluates the FMA-corrected quotient two lanes at a time with the reciprocal negated, which
+must give exactly the negated quotient (signed zeros included). This checks, on the CPU,
 that the identities hold on the domains the kernels use them on (a strided subset here;
-the exhaustive run, stride 1, also passes)."""
+the exhaustive run, stride 1, also passes for the first four)."""
 import os
 import subprocess
 
