@@ -273,7 +273,7 @@ struct QuantSmem {
   static constexpr int kVRowBytes = (D + 8) * 2;     // padded V tile row (16-byte multiple)
   static constexpr int kStats = kRG * D * 8 + 2 * kRG * D * 4 + (kThreads / 32) * 4;
   static constexpr int kVt = 128 * kVRowBytes + 1024;
-  static constexpr int kRows = 1024 + D * 4;
+  static constexpr int kRows = (D / 64) * 512;  // the Q / K tile's scale tile
 };
 
 // Statistics job (split, h, b): chunk `split` of sequence b, head h.
