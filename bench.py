@@ -55,6 +55,17 @@ def fp4_peak(peaks: dict, basis: str, probe=None, b8: bool = False):
     return peak, how
 
 
+def quant_algorithmic_bytes(wl, b8=False):
+    """Bytes the quantization of a dense problem with K smoothing must move: Q, K and V
+    read once, K read again after its mean (8-bit: V again after its channel scales), and
+    the quantized tensors written (FP4: half a byte per element plus one scale byte per 16
+    elements; 8-bit: one byte per element, scales negligible). 2-byte inputs."""
+    E = wl.B * wl.H * wl.N * wl.D
+    if b8:
+        return 5 * E * 2 + 3 * E
+    return 4 * E * 2 + 3 * E * (0.5 + 1.0 / 16.0)
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -620,6 +631,12 @@ def main():
         "fp4_mma_probe_tflops": None if probe is None else probe["tflops"],
         "attn_ms": attn_avg_ms, "quant_ms": statistics.mean(quant_ms),
     }
+    # The quantization's own HBM roofline: algorithmic bytes over its CUDA-event time.
+    qbytes = quant_algorithmic_bytes(wl, b8)
+    qgbs = qbytes / (roofline["quant_ms"] * 1e-3) / 1e9 if roofline["quant_ms"] > 0 else None
+    roofline["quant_bytes"] = qbytes
+    roofline["quant_gbs"] = qgbs
+    roofline["quant_frac_of_hbm"] = None if qgbs is None else qgbs / float(peaks.get("hbm_gbs", 6650.0))
     cpu = None
     if not args.no_cpu_baseline:
         val, _, sample, cores = cpu_oracle_rate(wl, args.cpu_budget_s)

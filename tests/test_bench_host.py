@@ -98,3 +98,14 @@ def test_committed_record_names_existing_sources(bench_mod):
         assert os.path.isfile(os.path.join(ROOT, s)), s
     t, src = bench_mod._attn_traffic(W.LONG)
     assert (t is not None and t > 0) or src == "kernel changed since the capture", src
+
+
+def test_quant_algorithmic_bytes_long_workload():
+    """The quantizer's algorithmic bytes for the long workload: Q, K, V read (604 MB), K
+    read again (201 MB), FP4 codes and scales written (170 MB) -- 975 MB."""
+    import bench
+    from microscaling_fp4_quantized_b200 import workloads as W
+    E = 24 * 32768 * 128
+    assert bench.quant_algorithmic_bytes(W.LONG) == 4 * E * 2 + 3 * E * 0.5625
+    assert abs(bench.quant_algorithmic_bytes(W.LONG) / 1e6 - 975.2) < 0.5
+    assert bench.quant_algorithmic_bytes(W.LONG, b8=True) == 13 * E
